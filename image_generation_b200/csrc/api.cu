@@ -1,0 +1,522 @@
+// C ABI of libh3dit (declared in include/h3dit.h): argument checks, the
+// workspace plan, TMA tensor-map encoding and the order of kernel launches
+// for one DiT block and one sampling step. All compute runs in the kernels of
+// gemm.cu, attention.cu and elementwise.cu; this file only marshals.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/h3dit.h"
+#include "kernels.h"
+
+using namespace h3;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Layout {
+  size_t status, resid, xm, qkv, attn, u, mod, cvec, hidden, rope, wptr, bptr, total;
+};
+
+bool config_ok(const h3dit_config *c) {
+  if (!c) return false;
+  if (c->hidden <= 0 || c->hidden % 64 || c->hidden > 8192) return false;
+  if (c->heads <= 0 || (c->head_dim != 96 && c->head_dim != 128)) return false;
+  if (c->ffn <= 0 || c->ffn % 64) return false;
+  if (c->n_blocks <= 0 || c->max_tokens <= 0) return false;
+  const int pairs = c->rope_sections[0] + c->rope_sections[1] + c->rope_sections[2];
+  if (2 * pairs != c->head_dim) return false;
+  for (int a = 0; a < 3; ++a)
+    if (c->rope_sections[a] != 16 && c->rope_sections[a] != 24) return false;
+  if (!(c->norm_eps >= 0.f) || !(c->rope_theta > 0.f)) return false;
+  if (c->precision != H3DIT_PRECISION_BF16 && c->precision != H3DIT_PRECISION_MXFP8) return false;
+  return true;
+}
+
+Layout plan(const h3dit_config *c) {
+  Layout L{};
+  const size_t N = static_cast<size_t>(c->max_tokens);
+  const size_t D = c->hidden, I = static_cast<size_t>(c->heads) * c->head_dim, F = c->ffn;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = round_up(off + bytes, kAlign);
+    return at;
+  };
+  L.status = take(kAlign);
+  L.resid = take(N * D * 4);
+  L.xm = take(N * D * 2);
+  L.qkv = take(N * 3 * I * 2);
+  L.attn = take(N * I * 2);
+  L.u = take(N * F * 2);
+  L.mod = take(static_cast<size_t>(c->n_blocks) * 6 * D * 4);
+  L.cvec = take(D * 4);
+  L.hidden = take(D * 4);
+  L.rope = take(N * (c->head_dim / 2) * 2 * 4);
+  L.wptr = take(static_cast<size_t>(c->n_blocks) * sizeof(void *));
+  L.bptr = take(static_cast<size_t>(c->n_blocks) * sizeof(void *));
+  L.total = off;
+  return L;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+struct h3dit_ctx {
+  h3dit_config cfg;
+  h3dit_time_weights tw;
+  std::vector<h3dit_block_weights> blocks;
+  uint8_t *ws = nullptr;
+  size_t ws_bytes = 0;
+  Layout L{};
+  int num_sms = 148;
+  std::string err;
+
+  int *status() { return reinterpret_cast<int *>(ws + L.status); }
+  float *resid() { return reinterpret_cast<float *>(ws + L.resid); }
+  void *xm() { return ws + L.xm; }
+  void *qkv() { return ws + L.qkv; }
+  void *attn() { return ws + L.attn; }
+  void *u() { return ws + L.u; }
+  float *mod(int l) { return reinterpret_cast<float *>(ws + L.mod) + static_cast<size_t>(l) * 6 * cfg.hidden; }
+  float *cvec() { return reinterpret_cast<float *>(ws + L.cvec); }
+  float *hidden() { return reinterpret_cast<float *>(ws + L.hidden); }
+  float *rope() { return reinterpret_cast<float *>(ws + L.rope); }
+  const void *const *wptr() { return reinterpret_cast<const void *const *>(ws + L.wptr); }
+  const float *const *bptr() { return reinterpret_cast<const float *const *>(ws + L.bptr); }
+  int inner() const { return cfg.heads * cfg.head_dim; }
+
+  h3dit_status fail(h3dit_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    err = buf;
+    return s;
+  }
+  h3dit_status cuda(cudaError_t e, const char *what) {
+    if (e == cudaSuccess) return H3DIT_OK;
+    return fail(H3DIT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  }
+};
+
+namespace {
+
+h3dit_status encode_2d(h3dit_ctx *ctx, CUtensorMap *m, const void *base, uint64_t inner,
+                       uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return ctx->fail(H3DIT_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return ctx->fail(H3DIT_ERR_CUDA, "tensor map encode failed (%d)", (int)r);
+  return H3DIT_OK;
+}
+
+// [tokens, heads, head_dim] view with a token stride of `ld` elements.
+h3dit_status encode_heads(h3dit_ctx *ctx, CUtensorMap *m, const void *base, int n, int heads,
+                          int head_dim, int ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return ctx->fail(H3DIT_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(n)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                                 static_cast<cuuint64_t>(ld) * 2};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return ctx->fail(H3DIT_ERR_CUDA, "tensor map encode failed (%d)", (int)r);
+  return H3DIT_OK;
+}
+
+h3dit_status run_linear(h3dit_ctx *ctx, int epi, const void *a, const void *w, int m, int n,
+                        int k, void *out, long long ldo, const float *gate, const float *rope,
+                        cudaStream_t s) {
+  if (epi < H3DIT_EPI_STORE || epi > H3DIT_EPI_GATED_RESIDUAL)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "unknown epilogue %d", epi);
+  if (m < 0 || n <= 0 || k <= 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "bad shape %d x %d x %d", m, n, k);
+  if (k % kGemmBK || n % 32)
+    return ctx->fail(H3DIT_ERR_UNSUPPORTED, "linear needs k %% 64 == 0 and n %% 32 == 0 (k=%d n=%d)", k, n);
+  if (!a || !w || !out || !aligned16(a) || !aligned16(w) || !aligned16(out))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "linear: NULL or misaligned pointer");
+  if (epi == H3DIT_EPI_GATED_RESIDUAL && (!gate || !aligned16(gate)))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "gated residual needs a 16-byte aligned gate");
+  GemmParams p{};
+  if (epi == H3DIT_EPI_QKV_ROPE) {
+    const int I = ctx->inner(), dh = ctx->cfg.head_dim;
+    const int *sec = ctx->cfg.rope_sections;
+    if (n != 3 * I) return ctx->fail(H3DIT_ERR_INVALID_ARG, "QKV epilogue needs n == 3*heads*head_dim");
+    if (!rope || !aligned16(rope)) return ctx->fail(H3DIT_ERR_INVALID_ARG, "QKV epilogue needs a RoPE table");
+    // each output tile must start on a rotary-section boundary of a head
+    for (int c = 0; c < 2 * I; c += kGemmBN) {
+      const int h = c % dh;
+      if (h != 0 && h != 2 * sec[0] && h != 2 * (sec[0] + sec[1]))
+        return ctx->fail(H3DIT_ERR_UNSUPPORTED, "rope sections do not align with 256-column tiles");
+    }
+    p.head_dim = dh;
+    p.rope_cols = 2 * I;
+    p.sec[0] = sec[0];
+    p.sec[1] = sec[1];
+    p.sec[2] = sec[2];
+  }
+  if (m == 0) return H3DIT_OK;
+  CUtensorMap ta, tb;
+  h3dit_status st = encode_2d(ctx, &ta, a, k, m, static_cast<uint64_t>(k) * 2, kGemmBK, kGemmBM);
+  if (st) return st;
+  st = encode_2d(ctx, &tb, w, k, n, static_cast<uint64_t>(k) * 2, kGemmBK, kGemmBN);
+  if (st) return st;
+  p.m = m;
+  p.n = n;
+  p.k = k;
+  p.tiles_m = (m + kGemmBM - 1) / kGemmBM;
+  p.tiles_n = (n + kGemmBN - 1) / kGemmBN;
+  p.out = out;
+  p.ldo = ldo;
+  p.gate = gate;
+  p.rope = rope;
+  p.gelu_tanh = ctx->cfg.gelu_tanh;
+  p.status = ctx->status();
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int grid = tiles < ctx->num_sms ? tiles : ctx->num_sms;
+  return ctx->cuda(launch_gemm(ta, tb, p, epi, grid, s), "gemm launch");
+}
+
+h3dit_status run_attention(h3dit_ctx *ctx, const void *q, const void *k, const void *v, int ld,
+                           void *o, int ldo, int n, cudaStream_t s) {
+  if (n < 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "n < 0");
+  if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "attention: NULL or misaligned pointer");
+  const int I = ctx->inner();
+  if (ld < I || ld % 8 || ldo < I || ldo % 8)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "attention: row strides must be >= heads*head_dim and multiples of 8");
+  if (n == 0) return H3DIT_OK;
+  CUtensorMap tq, tk, tv;
+  h3dit_status st;
+  if ((st = encode_heads(ctx, &tq, q, n, ctx->cfg.heads, ctx->cfg.head_dim, ld))) return st;
+  if ((st = encode_heads(ctx, &tk, k, n, ctx->cfg.heads, ctx->cfg.head_dim, ld))) return st;
+  if ((st = encode_heads(ctx, &tv, v, n, ctx->cfg.heads, ctx->cfg.head_dim, ld))) return st;
+  AttnParams p{};
+  p.n = n;
+  p.tiles_kv = (n + 127) / 128;
+  p.o = o;
+  p.ldo = ldo;
+  p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(ctx->cfg.head_dim));
+  p.status = ctx->status();
+  return ctx->cuda(launch_attention(tq, tk, tv, p, ctx->cfg.head_dim, ctx->cfg.heads, s),
+                   "attention launch");
+}
+
+h3dit_status check_tokens(h3dit_ctx *ctx, void *x_img, const h3dit_grid *grids, int n_grids,
+                          void *x_txt, int n_txt, int *n_img_out) {
+  if (n_txt < 0 || n_grids < 0 || n_grids > kMaxGrids)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "bad n_txt or n_grids (max %d grids)", kMaxGrids);
+  if (n_grids > 0 && !grids) return ctx->fail(H3DIT_ERR_INVALID_ARG, "grids is NULL");
+  long long n_img = 0;
+  for (int g = 0; g < n_grids; ++g) {
+    if (grids[g].height <= 0 || grids[g].width <= 0 || grids[g].frame < 0)
+      return ctx->fail(H3DIT_ERR_INVALID_ARG, "grid %d has a bad shape", g);
+    n_img += static_cast<long long>(grids[g].height) * grids[g].width;
+  }
+  const long long n = n_img + n_txt;
+  if (n < 1 || n > ctx->cfg.max_tokens)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "token count %lld outside [1, max_tokens=%d]", n, ctx->cfg.max_tokens);
+  if (n_img > 0 && (!x_img || !aligned16(x_img)))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "x_img is NULL or misaligned");
+  if (n_txt > 0 && (!x_txt || !aligned16(x_txt)))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "x_txt is NULL or misaligned");
+  *n_img_out = static_cast<int>(n_img);
+  return H3DIT_OK;
+}
+
+h3dit_status rope_table_into(h3dit_ctx *ctx, const h3dit_grid *grids, int n_grids, int n_txt,
+                             int n, float *table, cudaStream_t s) {
+  GridDesc g[kMaxGrids];
+  for (int i = 0; i < n_grids; ++i) g[i] = GridDesc{grids[i].frame, grids[i].height, grids[i].width};
+  return ctx->cuda(launch_rope_table(g, n_grids, n_txt, n, ctx->cfg.rope_sections,
+                                     ctx->cfg.rope_theta, table, s),
+                   "rope table launch");
+}
+
+// Steps a3..a9 on the packed fp32 residual of n tokens (workspace).
+h3dit_status block_body(h3dit_ctx *ctx, int l, const float *mod, int n, cudaStream_t s) {
+  const h3dit_block_weights &w = ctx->blocks[l];
+  const int D = ctx->cfg.hidden, I = ctx->inner(), F = ctx->cfg.ffn;
+  const float *sh1 = mod, *sc1 = mod + D, *g1 = mod + 2 * D;
+  const float *sh2 = mod + 3 * D, *sc2 = mod + 4 * D, *g2 = mod + 5 * D;
+  h3dit_status st;
+  if ((st = ctx->cuda(launch_rmsnorm_modulate(ctx->resid(), sh1, sc1, ctx->xm(), n, D,
+                                              ctx->cfg.norm_eps, ctx->num_sms, s),
+                      "rmsnorm launch")))
+    return st;
+  if ((st = run_linear(ctx, H3DIT_EPI_QKV_ROPE, ctx->xm(), w.w_qkv, n, 3 * I, D, ctx->qkv(), 3 * I,
+                       nullptr, ctx->rope(), s)))
+    return st;
+  const uint16_t *qkv = static_cast<const uint16_t *>(ctx->qkv());
+  if ((st = run_attention(ctx, qkv, qkv + I, qkv + 2 * I, 3 * I, ctx->attn(), I, n, s))) return st;
+  if ((st = run_linear(ctx, H3DIT_EPI_GATED_RESIDUAL, ctx->attn(), w.w_o, n, D, I, ctx->resid(), D,
+                       g1, nullptr, s)))
+    return st;
+  if ((st = ctx->cuda(launch_rmsnorm_modulate(ctx->resid(), sh2, sc2, ctx->xm(), n, D,
+                                              ctx->cfg.norm_eps, ctx->num_sms, s),
+                      "rmsnorm launch")))
+    return st;
+  if ((st = run_linear(ctx, H3DIT_EPI_GELU, ctx->xm(), w.w_ff1, n, F, D, ctx->u(), F, nullptr,
+                       nullptr, s)))
+    return st;
+  return run_linear(ctx, H3DIT_EPI_GATED_RESIDUAL, ctx->u(), w.w_ff2, n, D, F, ctx->resid(), D, g2,
+                    nullptr, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *h3dit_status_string(h3dit_status s) {
+  switch (s) {
+    case H3DIT_OK: return "ok";
+    case H3DIT_ERR_INVALID_ARG: return "invalid argument";
+    case H3DIT_ERR_UNSUPPORTED: return "unsupported shape or configuration";
+    case H3DIT_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case H3DIT_ERR_CUDA: return "CUDA error";
+    case H3DIT_ERR_TIMEOUT: return "a kernel's bounded wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char *h3dit_last_error(const h3dit_ctx *ctx) {
+  if (!ctx) return "no context";
+  return ctx->err.c_str();
+}
+
+size_t h3dit_workspace_bytes(const h3dit_config *cfg) {
+  if (!config_ok(cfg)) return 0;
+  return plan(cfg).total;
+}
+
+h3dit_status h3dit_create(const h3dit_config *cfg, const h3dit_time_weights *time_w,
+                          const h3dit_block_weights *blocks, void *workspace, size_t ws_bytes,
+                          void *cuda_stream, h3dit_ctx **out) {
+  if (!out) return H3DIT_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!config_ok(cfg) || !time_w || !blocks) return H3DIT_ERR_INVALID_ARG;
+  if (cfg->precision != H3DIT_PRECISION_BF16) return H3DIT_ERR_UNSUPPORTED;
+  if (!time_w->w_t1 || !time_w->b_t1 || !time_w->w_t2 || !time_w->b_t2 ||
+      !aligned16(time_w->w_t2))
+    return H3DIT_ERR_INVALID_ARG;
+  for (int l = 0; l < cfg->n_blocks; ++l) {
+    const h3dit_block_weights &b = blocks[l];
+    if (!b.w_qkv || !b.w_o || !b.w_ff1 || !b.w_ff2 || !b.w_ada || !b.b_ada) return H3DIT_ERR_INVALID_ARG;
+    if (!aligned16(b.w_qkv) || !aligned16(b.w_o) || !aligned16(b.w_ff1) || !aligned16(b.w_ff2) ||
+        !aligned16(b.w_ada))
+      return H3DIT_ERR_INVALID_ARG;
+  }
+  const Layout L = plan(cfg);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) || ws_bytes < L.total)
+    return H3DIT_ERR_WORKSPACE;
+
+  h3dit_ctx *ctx = new (std::nothrow) h3dit_ctx();
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  ctx->cfg = *cfg;
+  ctx->tw = *time_w;
+  ctx->blocks.assign(blocks, blocks + cfg->n_blocks);
+  ctx->ws = static_cast<uint8_t *>(workspace);
+  ctx->ws_bytes = ws_bytes;
+  ctx->L = L;
+  int dev = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    delete ctx;
+    return H3DIT_ERR_CUDA;
+  }
+  std::vector<const void *> wp(cfg->n_blocks), bp(cfg->n_blocks);
+  for (int l = 0; l < cfg->n_blocks; ++l) {
+    wp[l] = blocks[l].w_ada;
+    bp[l] = blocks[l].b_ada;
+  }
+  cudaError_t e = cudaMemsetAsync(ctx->status(), 0, sizeof(int), s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(ctx->ws + L.wptr, wp.data(), wp.size() * sizeof(void *),
+                        cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(ctx->ws + L.bptr, bp.data(), bp.size() * sizeof(void *),
+                        cudaMemcpyHostToDevice, s);
+  // the host vectors die with this call: the copies must have been consumed
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    delete ctx;
+    return H3DIT_ERR_CUDA;
+  }
+  *out = ctx;
+  return H3DIT_OK;
+}
+
+void h3dit_destroy(h3dit_ctx *ctx) { delete ctx; }
+
+h3dit_status h3dit_sync_status(h3dit_ctx *ctx, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return ctx->cuda(e, "stream synchronize");
+  int dev_status = 0;
+  e = cudaMemcpy(&dev_status, ctx->status(), sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return ctx->cuda(e, "status read");
+  if (dev_status != 0) {
+    cudaMemset(ctx->status(), 0, sizeof(int));
+    return ctx->fail(H3DIT_ERR_TIMEOUT, "a kernel's bounded wait gave up (device status %d)", dev_status);
+  }
+  return H3DIT_OK;
+}
+
+h3dit_status h3dit_time_embed(h3dit_ctx *ctx, float t, float *c_out, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (!c_out) return ctx->fail(H3DIT_ERR_INVALID_ARG, "c_out is NULL");
+  const h3dit_time_weights &w = ctx->tw;
+  return ctx->cuda(launch_time_embed(t, ctx->cfg.t_scale, w.w_t1, w.b_t1, w.w_t2, w.b_t2,
+                                     ctx->hidden(), c_out, ctx->cfg.hidden, ctx->status(),
+                                     static_cast<cudaStream_t>(cuda_stream)),
+                   "time embed launch");
+}
+
+h3dit_status h3dit_adaln_project(h3dit_ctx *ctx, const float *c, int32_t first, int32_t count,
+                                 float *mod_out, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (!c || !mod_out) return ctx->fail(H3DIT_ERR_INVALID_ARG, "NULL pointer");
+  if (first < 0 || count < 0 || first + count > ctx->cfg.n_blocks)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "block range [%d, %d) outside [0, %d)", first,
+                     first + count, ctx->cfg.n_blocks);
+  if (count == 0) return H3DIT_OK;
+  return ctx->cuda(launch_adaln(c, ctx->wptr(), ctx->bptr(), first, count, mod_out,
+                                ctx->cfg.hidden, ctx->num_sms,
+                                static_cast<cudaStream_t>(cuda_stream)),
+                   "adaln launch");
+}
+
+h3dit_status h3dit_rmsnorm_modulate(h3dit_ctx *ctx, const float *x, const float *shift,
+                                    const float *scale, void *xm_out, int32_t n,
+                                    void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (n < 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "n < 0");
+  if (!x || !shift || !scale || !xm_out || !aligned16(x) || !aligned16(shift) ||
+      !aligned16(scale) || !aligned16(xm_out))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "NULL or misaligned pointer");
+  if (n == 0) return H3DIT_OK;
+  return ctx->cuda(launch_rmsnorm_modulate(x, shift, scale, xm_out, n, ctx->cfg.hidden,
+                                           ctx->cfg.norm_eps, ctx->num_sms,
+                                           static_cast<cudaStream_t>(cuda_stream)),
+                   "rmsnorm launch");
+}
+
+h3dit_status h3dit_rope_table(h3dit_ctx *ctx, const h3dit_grid *grids, int32_t n_grids,
+                              int32_t n_txt, float *table_out, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (!table_out) return ctx->fail(H3DIT_ERR_INVALID_ARG, "table_out is NULL");
+  if (n_txt < 0 || n_grids < 0 || n_grids > kMaxGrids || (n_grids > 0 && !grids))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "bad grids");
+  long long n = n_txt;
+  for (int g = 0; g < n_grids; ++g) {
+    if (grids[g].height <= 0 || grids[g].width <= 0 || grids[g].frame < 0)
+      return ctx->fail(H3DIT_ERR_INVALID_ARG, "grid %d has a bad shape", g);
+    n += static_cast<long long>(grids[g].height) * grids[g].width;
+  }
+  if (n == 0) return H3DIT_OK;
+  if (n > (1LL << 30)) return ctx->fail(H3DIT_ERR_INVALID_ARG, "too many tokens");
+  return rope_table_into(ctx, grids, n_grids, n_txt, static_cast<int>(n), table_out,
+                         static_cast<cudaStream_t>(cuda_stream));
+}
+
+h3dit_status h3dit_linear(h3dit_ctx *ctx, int32_t epilogue, const void *a, const void *w,
+                          int32_t m, int32_t n, int32_t k, void *out, const float *gate,
+                          const float *rope_table, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  return run_linear(ctx, epilogue, a, w, m, n, k, out, n, gate, rope_table,
+                    static_cast<cudaStream_t>(cuda_stream));
+}
+
+h3dit_status h3dit_attention(h3dit_ctx *ctx, const void *q, const void *k, const void *v,
+                             int32_t ld_qkv, void *o, int32_t ld_o, int32_t n,
+                             void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  return run_attention(ctx, q, k, v, ld_qkv, o, ld_o, n, static_cast<cudaStream_t>(cuda_stream));
+}
+
+h3dit_status h3dit_block_forward(h3dit_ctx *ctx, int32_t block, float t, const float *mod,
+                                 void *x_img, const h3dit_grid *grids, int32_t n_grids,
+                                 void *x_txt, int32_t n_txt, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (block < 0 || block >= ctx->cfg.n_blocks)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "block %d outside [0, %d)", block, ctx->cfg.n_blocks);
+  if (mod && !aligned16(mod)) return ctx->fail(H3DIT_ERR_INVALID_ARG, "mod is misaligned");
+  int n_img = 0;
+  h3dit_status st = check_tokens(ctx, x_img, grids, n_grids, x_txt, n_txt, &n_img);
+  if (st) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  const int n = n_txt + n_img;
+  if ((st = rope_table_into(ctx, grids, n_grids, n_txt, n, ctx->rope(), s))) return st;
+  if (!mod) {
+    if ((st = h3dit_time_embed(ctx, t, ctx->cvec(), s))) return st;
+    if ((st = h3dit_adaln_project(ctx, ctx->cvec(), block, 1, ctx->mod(block), s))) return st;
+    mod = ctx->mod(block);
+  }
+  if ((st = ctx->cuda(launch_pack(x_txt, n_txt, x_img, n_img, ctx->cfg.hidden, ctx->resid(), s),
+                      "pack launch")))
+    return st;
+  if ((st = block_body(ctx, block, mod, n, s))) return st;
+  return ctx->cuda(launch_unpack(ctx->resid(), n_txt, n_img, ctx->cfg.hidden, x_txt, x_img, s),
+                   "unpack launch");
+}
+
+h3dit_status h3dit_step(h3dit_ctx *ctx, float t, void *x_img, const h3dit_grid *grids,
+                        int32_t n_grids, void *x_txt, int32_t n_txt, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  int n_img = 0;
+  h3dit_status st = check_tokens(ctx, x_img, grids, n_grids, x_txt, n_txt, &n_img);
+  if (st) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  const int n = n_txt + n_img;
+  if ((st = rope_table_into(ctx, grids, n_grids, n_txt, n, ctx->rope(), s))) return st;
+  if ((st = h3dit_time_embed(ctx, t, ctx->cvec(), s))) return st;
+  if ((st = h3dit_adaln_project(ctx, ctx->cvec(), 0, ctx->cfg.n_blocks, ctx->mod(0), s))) return st;
+  if ((st = ctx->cuda(launch_pack(x_txt, n_txt, x_img, n_img, ctx->cfg.hidden, ctx->resid(), s),
+                      "pack launch")))
+    return st;
+  for (int l = 0; l < ctx->cfg.n_blocks; ++l)
+    if ((st = block_body(ctx, l, ctx->mod(l), n, s))) return st;
+  return ctx->cuda(launch_unpack(ctx->resid(), n_txt, n_img, ctx->cfg.hidden, x_txt, x_img, s),
+                   "unpack launch");
+}
+
+}  // extern "C"

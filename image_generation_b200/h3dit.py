@@ -1,0 +1,222 @@
+"""ctypes binding of libh3dit (include/h3dit.h), same names as the C ABI.
+
+Argument marshalling only: every step of the block runs in the CUDA kernels of
+libh3dit.so. There is no fallback: if the library is missing, importing the
+binding raises. PyTorch is used by the helpers at the bottom only to hold
+device memory and to name the current CUDA stream.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import re
+from typing import List, Sequence, Tuple
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libh3dit.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "h3dit.h")
+
+H3DIT_OK = 0
+H3DIT_ERR_INVALID_ARG = -1
+H3DIT_ERR_UNSUPPORTED = -2
+H3DIT_ERR_WORKSPACE = -3
+H3DIT_ERR_CUDA = -4
+H3DIT_ERR_TIMEOUT = -5
+
+H3DIT_EPI_STORE = 0
+H3DIT_EPI_QKV_ROPE = 1
+H3DIT_EPI_GELU = 2
+H3DIT_EPI_GATED_RESIDUAL = 3
+
+H3DIT_PRECISION_BF16 = 0
+H3DIT_PRECISION_MXFP8 = 1
+
+
+class h3dit_config(C.Structure):
+    _fields_ = [
+        ("hidden", C.c_int32), ("heads", C.c_int32), ("head_dim", C.c_int32),
+        ("ffn", C.c_int32), ("n_blocks", C.c_int32), ("max_tokens", C.c_int32),
+        ("rope_sections", C.c_int32 * 3), ("rope_theta", C.c_float),
+        ("norm_eps", C.c_float), ("t_scale", C.c_float), ("gelu_tanh", C.c_int32),
+        ("precision", C.c_int32),
+    ]
+
+
+class h3dit_time_weights(C.Structure):
+    _fields_ = [("w_t1", C.c_void_p), ("b_t1", C.c_void_p), ("w_t2", C.c_void_p),
+                ("b_t2", C.c_void_p)]
+
+
+class h3dit_block_weights(C.Structure):
+    _fields_ = [("w_qkv", C.c_void_p), ("w_o", C.c_void_p), ("w_ff1", C.c_void_p),
+                ("w_ff2", C.c_void_p), ("w_ada", C.c_void_p), ("b_ada", C.c_void_p)]
+
+
+class h3dit_grid(C.Structure):
+    _fields_ = [("frame", C.c_int32), ("height", C.c_int32), ("width", C.c_int32)]
+
+
+class H3DitError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"h3dit status {status}: {msg}")
+        self.status = status
+
+
+def _load() -> C.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m image_generation_b200.build`")
+    lib = C.CDLL(LIB_PATH)
+    p, i32, f32, sz = C.c_void_p, C.c_int32, C.c_float, C.c_size_t
+    sig = {
+        "h3dit_status_string": (C.c_char_p, [i32]),
+        "h3dit_last_error": (C.c_char_p, [p]),
+        "h3dit_workspace_bytes": (sz, [C.POINTER(h3dit_config)]),
+        "h3dit_create": (i32, [C.POINTER(h3dit_config), C.POINTER(h3dit_time_weights),
+                               C.POINTER(h3dit_block_weights), p, sz, p, C.POINTER(p)]),
+        "h3dit_destroy": (None, [p]),
+        "h3dit_block_forward": (i32, [p, i32, f32, p, p, C.POINTER(h3dit_grid), i32, p, i32, p]),
+        "h3dit_step": (i32, [p, f32, p, C.POINTER(h3dit_grid), i32, p, i32, p]),
+        "h3dit_sync_status": (i32, [p, p]),
+        "h3dit_time_embed": (i32, [p, f32, p, p]),
+        "h3dit_adaln_project": (i32, [p, p, i32, i32, p, p]),
+        "h3dit_rmsnorm_modulate": (i32, [p, p, p, p, p, i32, p]),
+        "h3dit_rope_table": (i32, [p, C.POINTER(h3dit_grid), i32, i32, p, p]),
+        "h3dit_linear": (i32, [p, i32, p, p, i32, i32, i32, p, p, p, p]),
+        "h3dit_attention": (i32, [p, p, p, p, i32, p, i32, i32, p]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def header_functions() -> List[str]:
+    """Names of the functions include/h3dit.h declares."""
+    with open(HEADER) as fh:
+        text = fh.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(h3dit_[a-z_0-9]+)\s*\(", text)))
+
+
+def status_string(s: int) -> str:
+    return lib.h3dit_status_string(s).decode()
+
+
+def check(ctx, status: int) -> None:
+    if status != H3DIT_OK:
+        msg = lib.h3dit_last_error(ctx).decode() if ctx else status_string(status)
+        raise H3DitError(status, msg or status_string(status))
+
+
+def make_config(hidden: int, heads: int, head_dim: int, ffn: int, n_blocks: int,
+                max_tokens: int, sections: Sequence[int] | None = None,
+                rope_theta: float = 10000.0, norm_eps: float = 1e-6, t_scale: float = 1000.0,
+                gelu_tanh: bool = False, precision: int = H3DIT_PRECISION_BF16) -> h3dit_config:
+    if sections is None:
+        sections = {96: (16, 16, 16), 128: (16, 24, 24)}.get(head_dim, (0, 0, 0))
+    return h3dit_config(hidden, heads, head_dim, ffn, n_blocks, max_tokens,
+                        (C.c_int32 * 3)(*sections), rope_theta, norm_eps, t_scale,
+                        int(gelu_tanh), precision)
+
+
+def grids_array(grids: Sequence[Tuple[int, int, int]]):
+    arr = (h3dit_grid * max(1, len(grids)))()
+    for i, (f, h, w) in enumerate(grids):
+        arr[i] = h3dit_grid(f, h, w)
+    return arr
+
+
+# ---------------------------------------------------------------- torch helpers
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    import torch
+
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+class Context:
+    """Owns one h3dit_ctx plus the torch tensors it borrows (weights, workspace)."""
+
+    def __init__(self, cfg: h3dit_config, time_w: dict, blocks: Sequence[dict], stream=None):
+        import torch
+
+        self.cfg = cfg
+        self._keep = [time_w, list(blocks)]
+        ws_bytes = lib.h3dit_workspace_bytes(C.byref(cfg))
+        if ws_bytes == 0:
+            raise H3DitError(H3DIT_ERR_INVALID_ARG, "invalid config")
+        self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        tw = h3dit_time_weights(_ptr(time_w["w_t1"]), _ptr(time_w["b_t1"]),
+                                _ptr(time_w["w_t2"]), _ptr(time_w["b_t2"]))
+        arr = (h3dit_block_weights * len(blocks))()
+        for i, b in enumerate(blocks):
+            arr[i] = h3dit_block_weights(_ptr(b["w_qkv"]), _ptr(b["w_o"]), _ptr(b["w_ff1"]),
+                                         _ptr(b["w_ff2"]), _ptr(b["w_ada"]), _ptr(b["b_ada"]))
+        handle = C.c_void_p()
+        st = lib.h3dit_create(C.byref(cfg), C.byref(tw), arr, self.workspace.data_ptr(),
+                              ws_bytes, _stream(stream), C.byref(handle))
+        check(None, st)
+        self.handle = handle
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            lib.h3dit_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        self.close()
+
+    def _check(self, st: int) -> None:
+        check(self.handle, st)
+
+    def sync_status(self, stream=None) -> int:
+        return lib.h3dit_sync_status(self.handle, _stream(stream))
+
+    def time_embed(self, t: float, c_out, stream=None) -> None:
+        self._check(lib.h3dit_time_embed(self.handle, t, _ptr(c_out), _stream(stream)))
+
+    def adaln_project(self, c, first: int, count: int, mod_out, stream=None) -> None:
+        self._check(lib.h3dit_adaln_project(self.handle, _ptr(c), first, count, _ptr(mod_out),
+                                            _stream(stream)))
+
+    def rmsnorm_modulate(self, x, shift, scale, xm_out, stream=None) -> None:
+        self._check(lib.h3dit_rmsnorm_modulate(self.handle, _ptr(x), _ptr(shift), _ptr(scale),
+                                               _ptr(xm_out), x.shape[0], _stream(stream)))
+
+    def rope_table(self, grids, n_txt: int, table_out, stream=None) -> None:
+        g = grids_array(grids)
+        self._check(lib.h3dit_rope_table(self.handle, g, len(grids), n_txt, _ptr(table_out),
+                                         _stream(stream)))
+
+    def linear(self, epilogue: int, a, w, out, gate=None, rope_table=None, stream=None) -> None:
+        m, k = a.shape
+        n = w.shape[0]
+        self._check(lib.h3dit_linear(self.handle, epilogue, _ptr(a), _ptr(w), m, n, k, _ptr(out),
+                                     _ptr(gate), _ptr(rope_table), _stream(stream)))
+
+    def attention(self, q, k, v, ld_qkv: int, o, ld_o: int, n: int, stream=None) -> None:
+        self._check(lib.h3dit_attention(self.handle, _ptr(q), _ptr(k), _ptr(v), ld_qkv, _ptr(o),
+                                        ld_o, n, _stream(stream)))
+
+    def block_forward(self, block: int, t: float, x_img, grids, x_txt, mod=None,
+                      stream=None) -> None:
+        g = grids_array(grids)
+        n_txt = 0 if x_txt is None else x_txt.shape[0]
+        self._check(lib.h3dit_block_forward(self.handle, block, t, _ptr(mod), _ptr(x_img), g,
+                                            len(grids), _ptr(x_txt), n_txt, _stream(stream)))
+
+    def step(self, t: float, x_img, grids, x_txt, stream=None) -> None:
+        g = grids_array(grids)
+        n_txt = 0 if x_txt is None else x_txt.shape[0]
+        self._check(lib.h3dit_step(self.handle, t, _ptr(x_img), g, len(grids), _ptr(x_txt),
+                                   n_txt, _stream(stream)))

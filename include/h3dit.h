@@ -1,0 +1,190 @@
+/*
+ * h3dit.h - C ABI of the B200 (sm_100a) DiT-block library for MiniMax-H3-Image.
+ *
+ * What it computes: the denoising forward of the dense single-stream DiT
+ * block, repeated over the blocks of one sampling step.
+ *   - MiniMax-H3-Image model card, "Model Architecture": text and image tokens
+ *     form one packed sequence through a single-stream transformer with
+ *     50 layers, hidden 5376, 56 heads, FFN 14336 and 3D multimodal RoPE;
+ *     BF16 weights, FP32 timestep layers.
+ *   - apxml "MiniMax H3 Image", "Architecture Diagram": per block, RMSNorm with
+ *     timestep scale/shift -> joint attention -> "+" -> RMSNorm with timestep
+ *     scale/shift -> GELU MLP -> "+".
+ *   - "H3-Image Day-0 Support: 4K in 0.87s with Vera Rubin", "Faster DiT":
+ *     the AdaLN conditioning projection is computed once and reused.
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer named "device" is CUDA device memory owned by the caller;
+ *     the library never frees it. bf16 tensors are passed as raw 16-bit
+ *     patterns (`void*`). Device pointers must be 16-byte aligned.
+ *   - Matrices are row-major. Weights use the nn.Linear layout [out, in].
+ *   - All work is enqueued on `cuda_stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and is asynchronous. No call synchronises except
+ *     h3dit_sync_status. Calls never abort or exit the process.
+ *   - A context is used from one host thread at a time; two calls on one
+ *     context must not overlap on the GPU (they share its workspace).
+ *   - On an error, nothing is enqueued (validation happens first) unless the
+ *     status is H3DIT_ERR_CUDA; h3dit_last_error(ctx) gives the message.
+ */
+#ifndef H3DIT_H
+#define H3DIT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t h3dit_status;
+#define H3DIT_OK 0
+#define H3DIT_ERR_INVALID_ARG (-1) /* a NULL, misaligned or out-of-range argument */
+#define H3DIT_ERR_UNSUPPORTED (-2) /* a shape or head_dim this build does not run */
+#define H3DIT_ERR_WORKSPACE (-3)   /* workspace too small or misaligned */
+#define H3DIT_ERR_CUDA (-4)        /* a CUDA runtime or launch error */
+#define H3DIT_ERR_TIMEOUT (-5)     /* a kernel's bounded wait gave up (see h3dit_sync_status) */
+
+/* Epilogues of h3dit_linear (steps a4, a6/a9, a8 of the block). */
+#define H3DIT_EPI_STORE 0          /* out bf16 [m, n] = a w^T                          */
+#define H3DIT_EPI_QKV_ROPE 1       /* as STORE, RoPE on columns < 2*heads*head_dim    */
+#define H3DIT_EPI_GELU 2           /* out bf16 [m, n] = GELU(a w^T)                    */
+#define H3DIT_EPI_GATED_RESIDUAL 3 /* out fp32 [m, n] += gate[col] * (a w^T)          */
+
+#define H3DIT_PRECISION_BF16 0
+#define H3DIT_PRECISION_MXFP8 1
+
+typedef struct h3dit_config {
+  int32_t hidden;           /* D, multiple of 64 (5376 for the model)                  */
+  int32_t heads;            /* H (56)                                                  */
+  int32_t head_dim;         /* d_h, 96 or 128 (the pages give both readings)           */
+  int32_t ffn;              /* F, multiple of 64 (14336)                               */
+  int32_t n_blocks;         /* L, blocks run by h3dit_step (50)                        */
+  int32_t max_tokens;       /* largest packed sequence any call will pass              */
+  int32_t rope_sections[3]; /* rotation pairs per (frame,row,col) axis; sum = d_h/2    */
+  float rope_theta;         /* RoPE base (10000)                                       */
+  float norm_eps;           /* RMSNorm epsilon (1e-6)                                  */
+  float t_scale;            /* sinusoid argument is t_scale * t (1000)                 */
+  int32_t gelu_tanh;        /* 0: exact erf GELU, 1: tanh approximation                */
+  int32_t precision;        /* H3DIT_PRECISION_BF16 (MXFP8: H3DIT_ERR_UNSUPPORTED)     */
+} h3dit_config;
+
+/* Timestep MLP, fp32, nn.Linear layout: Linear(256 -> D), SiLU, Linear(D -> D). */
+typedef struct h3dit_time_weights {
+  const float *w_t1; /* device [D, 256] */
+  const float *b_t1; /* device [D]      */
+  const float *w_t2; /* device [D, D]   */
+  const float *b_t2; /* device [D]      */
+} h3dit_time_weights;
+
+/* One block's weights (bf16 unless noted), borrowed for the context's life. */
+typedef struct h3dit_block_weights {
+  const void *w_qkv;  /* device [3I, D]; rows [Q heads | K heads | V heads], I = H*d_h    */
+  const void *w_o;    /* device [D, I]                                                   */
+  const void *w_ff1;  /* device [F, D]                                                   */
+  const void *w_ff2;  /* device [D, F]                                                   */
+  const void *w_ada;  /* device [6D, D]; chunks shift1,scale1,gate1,shift2,scale2,gate2  */
+  const float *b_ada; /* device fp32 [6D]                                                */
+} h3dit_block_weights;
+
+/* One latent image in the packed sequence: its RoPE frame index and grid.
+ * Image tokens are row-major over (height, width). The target is frame 0;
+ * reference image k is frame k. Text tokens sit at position (0, 0, 0). */
+typedef struct h3dit_grid {
+  int32_t frame, height, width;
+} h3dit_grid;
+
+typedef struct h3dit_ctx h3dit_ctx;
+
+/* Name of a status code (static string). */
+const char *h3dit_status_string(h3dit_status s);
+
+/* Last error message of a context ("" if none; static text if ctx is NULL). */
+const char *h3dit_last_error(const h3dit_ctx *ctx);
+
+/* Bytes of device workspace h3dit_create needs for `cfg`, or 0 if `cfg` is
+ * invalid. It covers the fp32 residual stream, the bf16 activations (xm,
+ * Q|K|V, attention output, FFN hidden), the per-step modulation table
+ * [n_blocks][6][D], the timestep vectors, the RoPE table and a status word. */
+size_t h3dit_workspace_bytes(const h3dit_config *cfg);
+
+/* Create a context. `blocks` points to cfg->n_blocks host structs whose device
+ * pointers must stay valid until h3dit_destroy. `workspace` is device memory of
+ * at least h3dit_workspace_bytes(cfg) bytes, 256-byte aligned, lent to the
+ * context for its life. Enqueues a small copy of the weight pointer table on
+ * `cuda_stream`. On error *out is set to NULL. */
+h3dit_status h3dit_create(const h3dit_config *cfg, const h3dit_time_weights *time_w,
+                          const h3dit_block_weights *blocks, void *workspace, size_t ws_bytes,
+                          void *cuda_stream, h3dit_ctx **out);
+
+/* Frees the host state of a context (NULL-safe). Device memory is the caller's. */
+void h3dit_destroy(h3dit_ctx *ctx);
+
+/* Run block `block` in place on the packed sequence [x_txt; images]:
+ *   x_txt  device bf16 [n_txt, D] (may be NULL when n_txt == 0), in/out;
+ *   x_img  device bf16 [sum h*w, D], in/out, images in `grids` order;
+ *   mod    device fp32 [6, D] modulation for this block, or NULL to compute it
+ *          from `t` (timestep MLP then this block's AdaLN projection).
+ * The residual stream is kept in fp32 inside the call; the result is rounded
+ * to bf16 once. Needs 1 <= n_txt + sum h*w <= max_tokens. */
+h3dit_status h3dit_block_forward(h3dit_ctx *ctx, int32_t block, float t, const float *mod,
+                                 void *x_img, const h3dit_grid *grids, int32_t n_grids,
+                                 void *x_txt, int32_t n_txt, void *cuda_stream);
+
+/* One sampling step in place: the timestep MLP and all n_blocks AdaLN
+ * projections once, then the n_blocks blocks in order with an fp32 residual
+ * stream, rounded to bf16 at the end. Arguments as in h3dit_block_forward. */
+h3dit_status h3dit_step(h3dit_ctx *ctx, float t, void *x_img, const h3dit_grid *grids,
+                        int32_t n_grids, void *x_txt, int32_t n_txt, void *cuda_stream);
+
+/* Synchronise `cuda_stream`, then read and clear the context's device status
+ * word. Returns H3DIT_ERR_TIMEOUT if a kernel's bounded wait gave up since the
+ * last call, H3DIT_ERR_CUDA on a CUDA error, else H3DIT_OK. */
+h3dit_status h3dit_sync_status(h3dit_ctx *ctx, void *cuda_stream);
+
+/* ---- The steps of the path, one entry point each (same kernels the block
+ * and step run; used to check and time each step on its own). ---------- */
+
+/* a1: c = W_t2 SiLU(W_t1 e(t) + b_t1) + b_t2 with e(t) the 256-channel
+ * sinusoid [cos | sin] of t_scale*t at frequencies 10000^(-i/128).
+ * c_out: device fp32 [D]. Uses the context workspace as scratch. */
+h3dit_status h3dit_time_embed(h3dit_ctx *ctx, float t, float *c_out, void *cuda_stream);
+
+/* a2: mod[l] = W_ada[l] SiLU(c) + b_ada[l] for blocks l in [first, first+count).
+ * c: device fp32 [D]; mod_out: device fp32 [count, 6, D]. */
+h3dit_status h3dit_adaln_project(h3dit_ctx *ctx, const float *c, int32_t first, int32_t count,
+                                 float *mod_out, void *cuda_stream);
+
+/* a3/a7: xm = x / sqrt(mean(x^2) + eps) * (1 + scale) + shift, per row.
+ * x: device fp32 [n, D]; shift, scale: device fp32 [D]; xm_out: device bf16 [n, D]. */
+h3dit_status h3dit_rmsnorm_modulate(h3dit_ctx *ctx, const float *x, const float *shift,
+                                    const float *scale, void *xm_out, int32_t n,
+                                    void *cuda_stream);
+
+/* RoPE table of the packed sequence: table_out device fp32 [n, d_h/2, 2]
+ * holding (cos, sin) of each rotation pair's angle, pairs ordered frame axis,
+ * row axis, col axis; n = n_txt + sum h*w. */
+h3dit_status h3dit_rope_table(h3dit_ctx *ctx, const h3dit_grid *grids, int32_t n_grids,
+                              int32_t n_txt, float *table_out, void *cuda_stream);
+
+/* a4/a6/a8/a9: acc = a w^T with a device bf16 [m, k], w device bf16 [n, k];
+ * k and n multiples of 64 and 32; then the epilogue (H3DIT_EPI_*):
+ *   STORE / GELU  out: device bf16 [m, n];
+ *   QKV_ROPE      out: device bf16 [m, n] with n = 3*heads*head_dim and
+ *                 rope_table the table of h3dit_rope_table for these m tokens;
+ *   GATED_RESIDUAL out: device fp32 [m, n], updated in place; gate: fp32 [n]. */
+h3dit_status h3dit_linear(h3dit_ctx *ctx, int32_t epilogue, const void *a, const void *w,
+                          int32_t m, int32_t n, int32_t k, void *out, const float *gate,
+                          const float *rope_table, void *cuda_stream);
+
+/* a5: O_h = softmax(Q_h K_h^T / sqrt(d_h)) V_h over all n tokens, no mask, for
+ * every head. q, k, v: device bf16 [n, heads, d_h] rows with row stride ld_qkv
+ * elements (the Q|K|V output of the QKV step has ld_qkv = 3*heads*d_h);
+ * o: device bf16 [n, heads*d_h] with row stride ld_o. */
+h3dit_status h3dit_attention(h3dit_ctx *ctx, const void *q, const void *k, const void *v,
+                             int32_t ld_qkv, void *o, int32_t ld_o, int32_t n,
+                             void *cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* H3DIT_H */

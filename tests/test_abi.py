@@ -1,0 +1,114 @@
+"""The C-ABI library loads and exports every function include/h3dit.h declares;
+host-side argument checks return their status codes. No compute call is made,
+so these run without a GPU."""
+import ctypes as C
+import subprocess
+
+import pytest
+
+from image_generation_b200 import h3dit as H
+
+
+def test_library_exports_every_declared_function():
+    declared = H.header_functions()
+    assert "h3dit_create" in declared and "h3dit_step" in declared
+    out = subprocess.run(["nm", "-D", "--defined-only", H.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [f for f in declared if f not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    for f in declared:
+        assert hasattr(H.lib, f)
+
+
+def test_status_strings():
+    for s in (H.H3DIT_OK, H.H3DIT_ERR_INVALID_ARG, H.H3DIT_ERR_UNSUPPORTED,
+              H.H3DIT_ERR_WORKSPACE, H.H3DIT_ERR_CUDA, H.H3DIT_ERR_TIMEOUT):
+        assert H.status_string(s) and H.status_string(s) != "unknown status"
+    assert H.status_string(12345) == "unknown status"
+
+
+def _cfg(**kw):
+    base = dict(hidden=5376, heads=56, head_dim=96, ffn=14336, n_blocks=50, max_tokens=16896)
+    base.update(kw)
+    return H.make_config(**base)
+
+
+def test_workspace_bytes_covers_the_plan():
+    cfg = _cfg()
+    ws = H.lib.h3dit_workspace_bytes(C.byref(cfg))
+    N, D, I, F, L = 16896, 5376, 5376, 14336, 50
+    need = N * D * 4 + N * D * 2 + N * 3 * I * 2 + N * I * 2 + N * F * 2 + L * 6 * D * 4
+    assert need <= ws <= need + 64 * 1024 * 1024
+    # head_dim 128 makes the attention width 7168
+    ws128 = H.lib.h3dit_workspace_bytes(C.byref(_cfg(head_dim=128)))
+    assert ws128 > ws
+
+
+@pytest.mark.parametrize("bad", [
+    dict(hidden=100), dict(head_dim=64), dict(ffn=1000), dict(n_blocks=0), dict(max_tokens=0),
+    dict(sections=(16, 16, 8)), dict(heads=0),
+])
+def test_invalid_configs_have_no_workspace(bad):
+    assert H.lib.h3dit_workspace_bytes(C.byref(_cfg(**bad))) == 0
+    assert H.lib.h3dit_workspace_bytes(None) == 0
+
+
+def _fake_weights(n_blocks):
+    fake = 0x10000  # 16-byte aligned, never dereferenced by the host-side checks
+    tw = H.h3dit_time_weights(fake, fake, fake, fake)
+    arr = (H.h3dit_block_weights * n_blocks)()
+    for i in range(n_blocks):
+        arr[i] = H.h3dit_block_weights(fake, fake, fake, fake, fake, fake)
+    return tw, arr
+
+
+def test_create_rejects_bad_arguments_before_touching_the_device():
+    cfg = _cfg(hidden=768, heads=8, ffn=2048, n_blocks=2, max_tokens=288)
+    tw, arr = _fake_weights(2)
+    out = C.c_void_p(1)
+    ws = H.lib.h3dit_workspace_bytes(C.byref(cfg))
+    # no workspace
+    assert H.lib.h3dit_create(C.byref(cfg), C.byref(tw), arr, None, ws, None, C.byref(out)) \
+        == H.H3DIT_ERR_WORKSPACE
+    assert out.value is None
+    # too small / misaligned workspace
+    assert H.lib.h3dit_create(C.byref(cfg), C.byref(tw), arr, 0x100000, ws - 1, None,
+                              C.byref(out)) == H.H3DIT_ERR_WORKSPACE
+    assert H.lib.h3dit_create(C.byref(cfg), C.byref(tw), arr, 0x100010, ws, None,
+                              C.byref(out)) == H.H3DIT_ERR_WORKSPACE
+    # NULL weights, misaligned weight, bad config, NULL out
+    assert H.lib.h3dit_create(C.byref(cfg), None, arr, 0x100000, ws, None, C.byref(out)) \
+        == H.H3DIT_ERR_INVALID_ARG
+    arr[1].w_o = 0x10002
+    assert H.lib.h3dit_create(C.byref(cfg), C.byref(tw), arr, 0x100000, ws, None,
+                              C.byref(out)) == H.H3DIT_ERR_INVALID_ARG
+    bad = _cfg(hidden=100)
+    assert H.lib.h3dit_create(C.byref(bad), C.byref(tw), arr, 0x100000, ws, None,
+                              C.byref(out)) == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_create(C.byref(cfg), C.byref(tw), arr, 0x100000, ws, None, None) \
+        == H.H3DIT_ERR_INVALID_ARG
+    # a precision this build does not run
+    mx = _cfg(hidden=768, heads=8, ffn=2048, n_blocks=2, max_tokens=288, precision=1)
+    tw, arr = _fake_weights(2)
+    assert H.lib.h3dit_create(C.byref(mx), C.byref(tw), arr, 0x100000, ws, None,
+                              C.byref(out)) == H.H3DIT_ERR_UNSUPPORTED
+
+
+def test_null_context_is_rejected_everywhere():
+    g = H.grids_array([(0, 2, 2)])
+    assert H.lib.h3dit_block_forward(None, 0, 0.5, None, 0x10000, g, 1, None, 0, None) \
+        == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_step(None, 0.5, 0x10000, g, 1, None, 0, None) == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_sync_status(None, None) == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_time_embed(None, 0.5, 0x10000, None) == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_adaln_project(None, 0x10000, 0, 1, 0x10000, None) == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_rmsnorm_modulate(None, 0x10000, 0x10000, 0x10000, 0x10000, 4, None) \
+        == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_rope_table(None, g, 1, 0, 0x10000, None) == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_linear(None, 0, 0x10000, 0x10000, 4, 32, 64, 0x10000, None, None, None) \
+        == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_attention(None, 0x10000, 0x10000, 0x10000, 768, 0x10000, 768, 4, None) \
+        == H.H3DIT_ERR_INVALID_ARG
+    H.lib.h3dit_destroy(None)  # NULL-safe
+    assert H.lib.h3dit_last_error(None) == b"no context"
