@@ -1,0 +1,517 @@
+#!/usr/bin/env python
+"""Benchmark: one 50-block denoising step of the MiniMax-H3-Image DiT at a
+4096^2 canvas (16,384 image tokens + 512 text tokens), through libh3dit.
+
+    python bench.py [--gpus N --steps K --warmup W] [--head-dim 96|128]
+    python bench.py --impl reference          # the CPU oracle on a bounded sample
+    python bench.py --only attention          # one kernel kind alone (for profilers)
+
+Rank 0 prints one JSON line. Multi-GPU runs are independent replicas (the
+step does not shard): every rank runs its own step on its own weights, the
+timed region is bracketed by barriers and the slowest rank's time is used.
+Weights are random-init bf16 (44 GB for 50 blocks at head_dim 96), generated
+on the device from a seed; all inputs are larger than L2, so no flush is
+needed between steps.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+D, H, F, L = 5376, 56, 14336, 50
+N_TXT, GRID = 512, 128
+N_TOK = N_TXT + GRID * GRID
+METRIC = "ms per 50-block 4096^2 denoise step"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="h3dit", choices=["h3dit", "reference"])
+    ap.add_argument("--head-dim", type=int, default=96, choices=[96, 128])
+    ap.add_argument("--only", default=None,
+                    choices=["attention", "qkv", "out_proj", "ffn1", "ffn2", "rmsnorm", "adaln"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def workload_name(dh: int) -> str:
+    return (f"50-block DiT denoise step, 4096^2 canvas: {GRID}x{GRID} image + {N_TXT} text "
+            f"tokens (joint {N_TOK}), hidden {D}, {H} heads x {dh}, GELU FFN {F}, bf16")
+
+
+def flops_per_launch(kind: str, n: int, dh: int) -> float:
+    I = H * dh
+    return {"qkv": 2.0 * n * D * 3 * I, "attention": 4.0 * n * n * I,
+            "out_proj": 2.0 * n * I * D, "ffn1": 2.0 * n * D * F,
+            "ffn2": 2.0 * n * F * D}.get(kind, 0.0)
+
+
+def bytes_per_launch(kind: str, n: int, dh: int, blocks: int = L) -> float:
+    """Algorithmic HBM bytes of the memory-bound kernels."""
+    return {"rmsnorm": n * D * (4 + 2) + 2 * D * 4,
+            "adaln": blocks * 6 * D * (D * 2 + 4 + 4) + D * 4,
+            "time_embed": (D * 256 + D * D + 3 * D) * 4,
+            "pack": n * D * (2 + 4), "rope_table": n * (dh // 2) * 8}.get(kind, 0.0)
+
+
+def step_flops(n: int, dh: int) -> float:
+    I = H * dh
+    return L * (8.0 * n * D * I + 4.0 * n * D * F + 4.0 * n * n * I)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            return json.load(fh), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def traffic_for(kind: str, dh: int):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the kernel source as it is now; else None."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{kind}_dh{dh}.txt")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as fh:
+        for line in fh:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+    src = fields.get("source")
+    if not src or "sha256" not in fields or "dram_bytes_per_launch" not in fields:
+        return None
+    with open(os.path.join(ROOT, src), "rb") as fh:
+        if hashlib.sha256(fh.read()).hexdigest() != fields["sha256"]:
+            return None
+    return float(fields["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        load = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- device setup
+
+def dist_info():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def make_model(dh: int, seed: int):
+    import torch
+
+    from image_generation_b200 import h3dit as Hb
+
+    I = H * dh
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+
+    def w(*shape, dtype=torch.bfloat16):
+        return (torch.randn(*shape, device="cuda", generator=g) * 0.02).to(dtype)
+
+    tw = {"w_t1": w(D, 256, dtype=torch.float32), "b_t1": torch.zeros(D, device="cuda"),
+          "w_t2": w(D, D, dtype=torch.float32), "b_t2": torch.zeros(D, device="cuda")}
+    blocks = [{"w_qkv": w(3 * I, D), "w_o": w(D, I), "w_ff1": w(F, D), "w_ff2": w(D, F),
+               "w_ada": w(6 * D, D), "b_ada": torch.zeros(6 * D, device="cuda")}
+              for _ in range(L)]
+    cfg = Hb.make_config(D, H, dh, F, L, N_TOK)
+    return Hb.Context(cfg, tw, blocks), tw, blocks
+
+
+def tokens(seed: int):
+    import torch
+
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    x_txt = torch.randn(N_TXT, D, device="cuda", generator=g).bfloat16()
+    x_img = torch.randn(GRID * GRID, D, device="cuda", generator=g).bfloat16()
+    return x_txt, x_img
+
+
+def timesteps(k: int):
+    return [1.0 - (i % 6) / 6.0 for i in range(k)]
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def oracle_sample(dh: int, rows_a: int = 8, rows_b: int = 40, seed: int = 0):
+    """Time the oracle on one block of the 4096^2 step for two query-row
+    samples (keys and values always over all tokens) and extrapolate linearly
+    to all rows and to the 50 blocks of a step, plus the per-step timestep MLP
+    and AdaLN projections. Returns (ms per step, description, threads)."""
+    import numpy as np
+
+    from image_generation_b200 import synth
+    from oracle import dit_block as O
+
+    dims = synth.Dims(D, H, dh, F)
+    cfg = O.config_for(D, H, dh, F)
+    w = synth.block_weights(dims, seed)
+    tw = synth.time_weights(dims, seed)
+    pos = O.token_positions(N_TXT, [(0, GRID, GRID)])
+    x = synth.tokens(N_TOK, D, seed, "x").astype(np.float64)
+    rng = np.random.default_rng(seed)
+    t0 = time.perf_counter()
+    c = O.timestep_condition(0.5, tw, cfg)
+    t_time = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    mod = O.adaln_modulation(c, w["w_ada"], w["b_ada"])
+    t_ada = time.perf_counter() - t0
+    times = []
+    for r in (rows_a, rows_b):
+        rows = np.sort(rng.choice(N_TOK, r, replace=False))
+        t0 = time.perf_counter()
+        O.block_forward(x, mod, w, pos, cfg, rows=rows)
+        times.append(time.perf_counter() - t0)
+    slope = max((times[1] - times[0]) / (rows_b - rows_a), 0.0)
+    fixed = max(times[0] - slope * rows_a, 0.0)
+    block_s = fixed + slope * N_TOK
+    step_ms = 1e3 * (t_time + L * t_ada + L * block_s)
+    threads = _blas_threads()
+    desc = (f"oracle (float64 numpy) on one block of the step for {rows_a} and {rows_b} query rows "
+            f"(K/V over all {N_TOK} tokens): {times[0]:.2f} s and {times[1]:.2f} s; "
+            f"extrapolated linearly to {N_TOK} rows and x{L} blocks, plus the timestep MLP "
+            f"({t_time * 1e3:.1f} ms) and {L} AdaLN projections ({t_ada * 1e3:.1f} ms each)")
+    return step_ms, desc, threads, sum(times) + t_time + t_ada
+
+
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------- arms
+
+def run_reference(args):
+    world, rank, _ = dist_info()
+    if rank != 0:
+        return 0
+    vals = []
+    desc, threads = "", 1
+    for _ in range(min(args.warmup, 1)):
+        oracle_sample(args.head_dim)
+    t_all = time.perf_counter()
+    for _ in range(args.steps):
+        v, desc, threads, _ = oracle_sample(args.head_dim)
+        vals.append(v)
+    wall = time.perf_counter() - t_all
+    value = sum(vals) / len(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "ms",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": min(args.warmup, 1),
+        "ms_per_step": round(value, 1), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, random-init weights)",
+        "config": {"workload": workload_name(args.head_dim), "n_blocks": L, "tokens": N_TOK,
+                   "head_dim": args.head_dim, "parallelism": "replicas",
+                   "l2": "inputs larger than L2"},
+        "cpu_baseline": {"value": round(value, 1), "unit": "ms", "cores": threads,
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 1), "unit": "ms", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "wall_s": round(wall, 1),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_only(args):
+    """One kernel kind alone at the step's shape (for ncu captures)."""
+    import torch
+
+    from image_generation_b200 import h3dit as Hb
+
+    dh = args.head_dim
+    I = H * dh
+    torch.manual_seed(0)
+    cfg = Hb.make_config(D, H, dh, F, 1, N_TOK)
+    g = lambda *s: (torch.randn(*s, device="cuda") * 0.02).bfloat16()
+    tw = {"w_t1": torch.randn(D, 256, device="cuda") * 0.02, "b_t1": torch.zeros(D, device="cuda"),
+          "w_t2": torch.randn(D, D, device="cuda") * 0.02, "b_t2": torch.zeros(D, device="cuda")}
+    need = {"qkv": "w_qkv", "out_proj": "w_o", "ffn1": "w_ff1", "ffn2": "w_ff2"}.get(args.only)
+    shapes = {"w_qkv": (3 * I, D), "w_o": (D, I), "w_ff1": (F, D), "w_ff2": (D, F), "w_ada": (6 * D, D)}
+    blk = {k: (g(*shp) if k in (need, "w_ada") else torch.zeros(8, device="cuda").bfloat16())
+           for k, shp in shapes.items()}
+    blk["b_ada"] = torch.zeros(6 * D, device="cuda")
+    ctx = Hb.Context(cfg, tw, [blk])
+    n = N_TOK
+    if args.only == "attention":
+        qkv = torch.randn(n, 3 * I, device="cuda").bfloat16()
+        o = torch.empty(n, I, device="cuda", dtype=torch.bfloat16)
+        fn = lambda: ctx.attention(qkv[:, :I], qkv[:, I:2 * I], qkv[:, 2 * I:], 3 * I, o, I, n)
+    elif args.only in ("qkv", "ffn1"):
+        xm = torch.randn(n, D, device="cuda").bfloat16()
+        table = torch.empty(n, dh // 2, 2, device="cuda")
+        ctx.rope_table([(0, GRID, GRID)], N_TXT, table)
+        out = torch.empty(n, blk[need].shape[0], device="cuda", dtype=torch.bfloat16)
+        epi = Hb.H3DIT_EPI_QKV_ROPE if args.only == "qkv" else Hb.H3DIT_EPI_GELU
+        fn = lambda: ctx.linear(epi, xm, blk[need], out, rope_table=table)
+    elif args.only in ("out_proj", "ffn2"):
+        a = torch.randn(n, blk[need].shape[1], device="cuda").bfloat16()
+        x = torch.randn(n, D, device="cuda")
+        gate = torch.full((D,), 0.1, device="cuda")
+        fn = lambda: ctx.linear(Hb.H3DIT_EPI_GATED_RESIDUAL, a, blk[need], x, gate=gate)
+    elif args.only == "rmsnorm":
+        x = torch.randn(n, D, device="cuda")
+        z = torch.zeros(D, device="cuda")
+        out = torch.empty(n, D, device="cuda", dtype=torch.bfloat16)
+        fn = lambda: ctx.rmsnorm_modulate(x, z, z, out)
+    else:  # adaln, one block
+        c = torch.randn(D, device="cuda")
+        mod = torch.empty(1, 6, D, device="cuda")
+        fn = lambda: ctx.adaln_project(c, 0, 1, mod)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    ctx.profile_begin()
+    for _ in range(args.steps):
+        fn()
+    prof = ctx.profile_end()
+    assert ctx.sync_status() == 0
+    ms, cnt = prof[args.only]
+    per = ms / max(cnt, 1)
+    fl = flops_per_launch(args.only, n, dh)
+    by = bytes_per_launch(args.only, n, dh, blocks=1)
+    out = {"kernel": args.only, "head_dim": dh, "tokens": n, "launches": cnt, "ms_per_launch": per}
+    if fl:
+        out["tflops"] = fl / per / 1e9
+    if by:
+        out["gbs"] = by / per / 1e6
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def run_h3dit(args):
+    import torch
+
+    world, rank, local = dist_info()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        dist = None
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    dh = args.head_dim
+    ctx, tw, blocks = make_model(dh, seed=1000 + rank)
+    x_txt, x_img = tokens(seed=rank)
+    grids = [(0, GRID, GRID)]
+    ts = timesteps(args.warmup + args.steps)
+
+    for i in range(args.warmup):
+        ctx.step(ts[i], x_img, grids, x_txt)
+    barrier()
+    st = ctx.sync_status()
+    if st != 0:
+        raise RuntimeError(f"warm-up failed with status {st}")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    ctx.profile_begin()
+    n0 = ctx.launch_count()
+    e0.record(stream)
+    for i in range(args.steps):
+        ctx.step(ts[args.warmup + i], x_img, grids, x_txt)
+    e1.record(stream)
+    barrier()
+    launches = ctx.launch_count() - n0
+    prof = ctx.profile_end()
+    clk = clocks.stop()
+    elapsed = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([elapsed], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+    st = ctx.sync_status()
+    if st != 0:
+        raise RuntimeError(f"timed steps failed with status {st}")
+    ms_step = elapsed / args.steps
+
+    # end to end: host (pinned) tokens in, step, tokens back to the host
+    e2e = None
+    if not args.no_e2e:
+        h_txt = torch.empty(x_txt.shape, dtype=x_txt.dtype, pin_memory=True)
+        h_img = torch.empty(x_img.shape, dtype=x_img.dtype, pin_memory=True)
+        h_txt.copy_(x_txt)
+        h_img.copy_(x_img)
+        o_txt = torch.empty_like(h_txt, pin_memory=True)
+        o_img = torch.empty_like(h_img, pin_memory=True)
+
+        def e2e_step(t):
+            x_txt.copy_(h_txt, non_blocking=True)
+            x_img.copy_(h_img, non_blocking=True)
+            ctx.step(t, x_img, grids, x_txt)
+            o_txt.copy_(x_txt, non_blocking=True)
+            o_img.copy_(x_img, non_blocking=True)
+
+        e2e_step(ts[0])
+        barrier()
+        e0.record(stream)
+        for i in range(args.steps):
+            e2e_step(ts[i])
+        e1.record(stream)
+        barrier()
+        e_ms = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([e_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        nbytes = (h_txt.numel() + h_img.numel()) * h_txt.element_size()
+        e2e = {"value": round(e_ms / args.steps / world, 2), "unit": "ms",
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
+        if ctx.sync_status() != 0:
+            raise RuntimeError("end-to-end steps failed")
+
+    line = None
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        dom = max((k for k in prof if prof[k][1] > 0), key=lambda k: prof[k][0])
+        ms_k, cnt_k = prof[dom]
+        per = ms_k / cnt_k
+        fl = flops_per_launch(dom, N_TOK, dh)
+        if fl:
+            achieved = fl / per / 1e9
+            peak = float(peaks["bf16_tflops_sustained"])
+            roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4)}
+        else:
+            achieved = bytes_per_launch(dom, N_TOK, dh) / per / 1e6
+            peak = float(peaks["hbm_gbs"])
+            roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                    "frac": round(achieved / peak, 4)}
+        roof.update({"kernel": dom, "ms_per_launch": round(per, 4), "launches": cnt_k,
+                     "peak_source": f"{peak_src} (sustained bf16)" if fl else f"{peak_src} (hbm copy)",
+                     "traffic": traffic_for(dom, dh)})
+        kernels = {}
+        for k, (ms, cnt) in prof.items():
+            if cnt == 0:
+                continue
+            ent = {"ms_total": round(ms, 3), "launches": cnt,
+                   "share": round(ms / max(sum(v[0] for v in prof.values()), 1e-9), 4)}
+            f = flops_per_launch(k, N_TOK, dh)
+            b = bytes_per_launch(k, N_TOK, dh)
+            if f:
+                ent["tflops"] = round(f / (ms / cnt) / 1e9, 1)
+            elif b:
+                ent["gbs"] = round(b / (ms / cnt) / 1e6, 1)
+            kernels[k] = ent
+        value = ms_step / world
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "ms", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 2),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded, random-init weights N(0,0.02), tokens N(0,1))",
+            "config": {"workload": workload_name(dh), "n_blocks": L, "tokens": N_TOK,
+                       "head_dim": dh, "global_batch": world,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (~44 GB of weights read per step)"},
+            "tflops_step": round(step_flops(N_TOK, dh) / ms_step / 1e9, 1),
+            "frac_of_bf16_peak_step": round(step_flops(N_TOK, dh) / ms_step / 1e9 /
+                                            float(peaks["bf16_tflops_sustained"]), 4),
+            "roofline": roof, "kernels": kernels, "gpu_launches": launches,
+            "e2e": e2e, "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            v, desc, threads, secs = oracle_sample(dh)
+            line["cpu_baseline"] = {"value": round(v, 1), "unit": "ms", "cores": threads,
+                                    "kind": "oracle", "sample": desc,
+                                    "sample_cpu_seconds": round(secs, 1)}
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.only:
+        return run_only(args)
+    return run_h3dit(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -37,6 +37,7 @@ bool config_ok(const h3dit_config *c) {
     if (c->rope_sections[a] != 16 && c->rope_sections[a] != 24) return false;
   if (!(c->norm_eps >= 0.f) || !(c->rope_theta > 0.f)) return false;
   if (c->precision != H3DIT_PRECISION_BF16 && c->precision != H3DIT_PRECISION_MXFP8) return false;
+  if (c->io_fp32 != 0 && c->io_fp32 != 1) return false;
   return true;
 }
 
@@ -88,8 +89,17 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 }  // namespace
 
+struct ProfRecord {
+  int kind;
+  cudaEvent_t begin, end;
+};
+
 struct h3dit_ctx {
   h3dit_config cfg;
+  bool profiling = false;
+  std::vector<ProfRecord> records;
+  std::vector<cudaEvent_t> event_pool;
+  long long launches = 0;
   h3dit_time_weights tw;
   std::vector<h3dit_block_weights> blocks;
   uint8_t *ws = nullptr;
@@ -125,7 +135,51 @@ struct h3dit_ctx {
     if (e == cudaSuccess) return H3DIT_OK;
     return fail(H3DIT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
   }
+  cudaEvent_t take_event() {
+    if (!event_pool.empty()) {
+      cudaEvent_t e = event_pool.back();
+      event_pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+  void recycle_records() {
+    for (auto &r : records) {
+      event_pool.push_back(r.begin);
+      event_pool.push_back(r.end);
+    }
+    records.clear();
+  }
+  ~h3dit_ctx() {
+    recycle_records();
+    for (cudaEvent_t e : event_pool) cudaEventDestroy(e);
+  }
 };
+
+namespace {
+// Counts the kernels of one library step and, while profiling, brackets them
+// with a CUDA event pair on the launch stream.
+struct Launch {
+  h3dit_ctx *ctx;
+  cudaStream_t s;
+  ProfRecord rec{};
+  bool on = false;
+  Launch(h3dit_ctx *c, int kind, cudaStream_t st, int kernels = 1) : ctx(c), s(st) {
+    ctx->launches += kernels;
+    if (ctx->profiling) {
+      rec.kind = kind;
+      rec.begin = ctx->take_event();
+      rec.end = ctx->take_event();
+      on = rec.begin && rec.end && cudaEventRecord(rec.begin, s) == cudaSuccess;
+    }
+  }
+  ~Launch() {
+    if (on && cudaEventRecord(rec.end, s) == cudaSuccess) ctx->records.push_back(rec);
+  }
+};
+}  // namespace
 
 namespace {
 
@@ -211,6 +265,12 @@ h3dit_status run_linear(h3dit_ctx *ctx, int epi, const void *a, const void *w, i
   p.status = ctx->status();
   const int tiles = p.tiles_m * p.tiles_n;
   const int grid = tiles < ctx->num_sms ? tiles : ctx->num_sms;
+  const int kind = epi == H3DIT_EPI_QKV_ROPE   ? H3DIT_KERNEL_QKV
+                   : epi == H3DIT_EPI_GELU     ? H3DIT_KERNEL_FFN1
+                   : k == ctx->inner()         ? H3DIT_KERNEL_OUT_PROJ
+                   : epi == H3DIT_EPI_STORE    ? H3DIT_KERNEL_FFN1
+                                               : H3DIT_KERNEL_FFN2;
+  Launch L(ctx, kind, s);
   return ctx->cuda(launch_gemm(ta, tb, p, epi, grid, s), "gemm launch");
 }
 
@@ -235,6 +295,7 @@ h3dit_status run_attention(h3dit_ctx *ctx, const void *q, const void *k, const v
   p.ldo = ldo;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(ctx->cfg.head_dim));
   p.status = ctx->status();
+  Launch L(ctx, H3DIT_KERNEL_ATTENTION, s);
   return ctx->cuda(launch_attention(tq, tk, tv, p, ctx->cfg.head_dim, ctx->cfg.heads, s),
                    "attention launch");
 }
@@ -265,9 +326,34 @@ h3dit_status rope_table_into(h3dit_ctx *ctx, const h3dit_grid *grids, int n_grid
                              int n, float *table, cudaStream_t s) {
   GridDesc g[kMaxGrids];
   for (int i = 0; i < n_grids; ++i) g[i] = GridDesc{grids[i].frame, grids[i].height, grids[i].width};
+  Launch L(ctx, H3DIT_KERNEL_ROPE_TABLE, s);
   return ctx->cuda(launch_rope_table(g, n_grids, n_txt, n, ctx->cfg.rope_sections,
                                      ctx->cfg.rope_theta, table, s),
                    "rope table launch");
+}
+
+h3dit_status run_rmsnorm(h3dit_ctx *ctx, const float *x, const float *shift, const float *scale,
+                         void *out, int n, cudaStream_t s) {
+  Launch L(ctx, H3DIT_KERNEL_RMSNORM, s);
+  return ctx->cuda(launch_rmsnorm_modulate(x, shift, scale, out, n, ctx->cfg.hidden,
+                                           ctx->cfg.norm_eps, ctx->num_sms, s),
+                   "rmsnorm launch");
+}
+
+h3dit_status run_pack(h3dit_ctx *ctx, const void *x_txt, int n_txt, const void *x_img, int n_img,
+                      cudaStream_t s) {
+  Launch L(ctx, H3DIT_KERNEL_PACK, s);
+  return ctx->cuda(launch_pack(x_txt, n_txt, x_img, n_img, ctx->cfg.hidden, ctx->cfg.io_fp32 != 0,
+                               ctx->resid(), s),
+                   "pack launch");
+}
+
+h3dit_status run_unpack(h3dit_ctx *ctx, int n_txt, int n_img, void *x_txt, void *x_img,
+                        cudaStream_t s) {
+  Launch L(ctx, H3DIT_KERNEL_PACK, s);
+  return ctx->cuda(launch_unpack(ctx->resid(), n_txt, n_img, ctx->cfg.hidden,
+                                 ctx->cfg.io_fp32 != 0, x_txt, x_img, s),
+                   "unpack launch");
 }
 
 // Steps a3..a9 on the packed fp32 residual of n tokens (workspace).
@@ -276,11 +362,8 @@ h3dit_status block_body(h3dit_ctx *ctx, int l, const float *mod, int n, cudaStre
   const int D = ctx->cfg.hidden, I = ctx->inner(), F = ctx->cfg.ffn;
   const float *sh1 = mod, *sc1 = mod + D, *g1 = mod + 2 * D;
   const float *sh2 = mod + 3 * D, *sc2 = mod + 4 * D, *g2 = mod + 5 * D;
-  h3dit_status st;
-  if ((st = ctx->cuda(launch_rmsnorm_modulate(ctx->resid(), sh1, sc1, ctx->xm(), n, D,
-                                              ctx->cfg.norm_eps, ctx->num_sms, s),
-                      "rmsnorm launch")))
-    return st;
+  h3dit_status st = run_rmsnorm(ctx, ctx->resid(), sh1, sc1, ctx->xm(), n, s);
+  if (st) return st;
   if ((st = run_linear(ctx, H3DIT_EPI_QKV_ROPE, ctx->xm(), w.w_qkv, n, 3 * I, D, ctx->qkv(), 3 * I,
                        nullptr, ctx->rope(), s)))
     return st;
@@ -289,10 +372,7 @@ h3dit_status block_body(h3dit_ctx *ctx, int l, const float *mod, int n, cudaStre
   if ((st = run_linear(ctx, H3DIT_EPI_GATED_RESIDUAL, ctx->attn(), w.w_o, n, D, I, ctx->resid(), D,
                        g1, nullptr, s)))
     return st;
-  if ((st = ctx->cuda(launch_rmsnorm_modulate(ctx->resid(), sh2, sc2, ctx->xm(), n, D,
-                                              ctx->cfg.norm_eps, ctx->num_sms, s),
-                      "rmsnorm launch")))
-    return st;
+  if ((st = run_rmsnorm(ctx, ctx->resid(), sh2, sc2, ctx->xm(), n, s))) return st;
   if ((st = run_linear(ctx, H3DIT_EPI_GELU, ctx->xm(), w.w_ff1, n, F, D, ctx->u(), F, nullptr,
                        nullptr, s)))
     return st;
@@ -405,6 +485,7 @@ h3dit_status h3dit_time_embed(h3dit_ctx *ctx, float t, float *c_out, void *cuda_
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
   if (!c_out) return ctx->fail(H3DIT_ERR_INVALID_ARG, "c_out is NULL");
   const h3dit_time_weights &w = ctx->tw;
+  Launch L(ctx, H3DIT_KERNEL_TIME_EMBED, static_cast<cudaStream_t>(cuda_stream), 2);
   return ctx->cuda(launch_time_embed(t, ctx->cfg.t_scale, w.w_t1, w.b_t1, w.w_t2, w.b_t2,
                                      ctx->hidden(), c_out, ctx->cfg.hidden, ctx->status(),
                                      static_cast<cudaStream_t>(cuda_stream)),
@@ -419,6 +500,7 @@ h3dit_status h3dit_adaln_project(h3dit_ctx *ctx, const float *c, int32_t first, 
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "block range [%d, %d) outside [0, %d)", first,
                      first + count, ctx->cfg.n_blocks);
   if (count == 0) return H3DIT_OK;
+  Launch L(ctx, H3DIT_KERNEL_ADALN, static_cast<cudaStream_t>(cuda_stream));
   return ctx->cuda(launch_adaln(c, ctx->wptr(), ctx->bptr(), first, count, mod_out,
                                 ctx->cfg.hidden, ctx->num_sms,
                                 static_cast<cudaStream_t>(cuda_stream)),
@@ -434,10 +516,7 @@ h3dit_status h3dit_rmsnorm_modulate(h3dit_ctx *ctx, const float *x, const float 
       !aligned16(scale) || !aligned16(xm_out))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "NULL or misaligned pointer");
   if (n == 0) return H3DIT_OK;
-  return ctx->cuda(launch_rmsnorm_modulate(x, shift, scale, xm_out, n, ctx->cfg.hidden,
-                                           ctx->cfg.norm_eps, ctx->num_sms,
-                                           static_cast<cudaStream_t>(cuda_stream)),
-                   "rmsnorm launch");
+  return run_rmsnorm(ctx, x, shift, scale, xm_out, n, static_cast<cudaStream_t>(cuda_stream));
 }
 
 h3dit_status h3dit_rope_table(h3dit_ctx *ctx, const h3dit_grid *grids, int32_t n_grids,
@@ -491,12 +570,9 @@ h3dit_status h3dit_block_forward(h3dit_ctx *ctx, int32_t block, float t, const f
     if ((st = h3dit_adaln_project(ctx, ctx->cvec(), block, 1, ctx->mod(block), s))) return st;
     mod = ctx->mod(block);
   }
-  if ((st = ctx->cuda(launch_pack(x_txt, n_txt, x_img, n_img, ctx->cfg.hidden, ctx->resid(), s),
-                      "pack launch")))
-    return st;
+  if ((st = run_pack(ctx, x_txt, n_txt, x_img, n_img, s))) return st;
   if ((st = block_body(ctx, block, mod, n, s))) return st;
-  return ctx->cuda(launch_unpack(ctx->resid(), n_txt, n_img, ctx->cfg.hidden, x_txt, x_img, s),
-                   "unpack launch");
+  return run_unpack(ctx, n_txt, n_img, x_txt, x_img, s);
 }
 
 h3dit_status h3dit_step(h3dit_ctx *ctx, float t, void *x_img, const h3dit_grid *grids,
@@ -510,13 +586,43 @@ h3dit_status h3dit_step(h3dit_ctx *ctx, float t, void *x_img, const h3dit_grid *
   if ((st = rope_table_into(ctx, grids, n_grids, n_txt, n, ctx->rope(), s))) return st;
   if ((st = h3dit_time_embed(ctx, t, ctx->cvec(), s))) return st;
   if ((st = h3dit_adaln_project(ctx, ctx->cvec(), 0, ctx->cfg.n_blocks, ctx->mod(0), s))) return st;
-  if ((st = ctx->cuda(launch_pack(x_txt, n_txt, x_img, n_img, ctx->cfg.hidden, ctx->resid(), s),
-                      "pack launch")))
-    return st;
+  if ((st = run_pack(ctx, x_txt, n_txt, x_img, n_img, s))) return st;
   for (int l = 0; l < ctx->cfg.n_blocks; ++l)
     if ((st = block_body(ctx, l, ctx->mod(l), n, s))) return st;
-  return ctx->cuda(launch_unpack(ctx->resid(), n_txt, n_img, ctx->cfg.hidden, x_txt, x_img, s),
-                   "unpack launch");
+  return run_unpack(ctx, n_txt, n_img, x_txt, x_img, s);
 }
+
+h3dit_status h3dit_profile_begin(h3dit_ctx *ctx) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  ctx->recycle_records();
+  ctx->profiling = true;
+  return H3DIT_OK;
+}
+
+h3dit_status h3dit_profile_end(h3dit_ctx *ctx, float *ms_out, int64_t *launches_out) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  ctx->profiling = false;
+  float ms[H3DIT_KERNEL_COUNT] = {};
+  int64_t cnt[H3DIT_KERNEL_COUNT] = {};
+  for (const ProfRecord &r : ctx->records) {
+    cudaError_t e = cudaEventSynchronize(r.end);
+    float t = 0.f;
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.begin, r.end);
+    if (e != cudaSuccess) {
+      ctx->recycle_records();
+      return ctx->cuda(e, "profile event");
+    }
+    ms[r.kind] += t;
+    cnt[r.kind] += 1;
+  }
+  ctx->recycle_records();
+  for (int k = 0; k < H3DIT_KERNEL_COUNT; ++k) {
+    if (ms_out) ms_out[k] = ms[k];
+    if (launches_out) launches_out[k] = cnt[k];
+  }
+  return H3DIT_OK;
+}
+
+int64_t h3dit_launch_count(const h3dit_ctx *ctx) { return ctx ? ctx->launches : 0; }
 
 }  // extern "C"

@@ -13,7 +13,7 @@
 namespace h3 {
 namespace {
 
-__device__ __forceinline__ float silu_f(float x) { return x / (1.f + __expf(-x)); }
+__device__ __forceinline__ float silu_f(float x) { return x / (1.f + expf(-x)); }
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -211,35 +211,48 @@ __global__ void rope_table_kernel(GridArray grids, int n_grids, int n_txt, int n
 }
 
 // ---------------------------------------------------------------- pack / unpack
-__global__ void pack_kernel(const uint16_t *__restrict__ x_txt, int n_txt,
-                            const uint16_t *__restrict__ x_img, int n_img, int d,
-                            float *__restrict__ resid) {
+// Four elements per thread-iteration; token buffers are bf16 or fp32.
+__device__ __forceinline__ float4 load4(const uint16_t *p, long long e) {
+  const uint2 v = *reinterpret_cast<const uint2 *>(p + e);
+  return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                     __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+}
+__device__ __forceinline__ float4 load4(const float *p, long long e) {
+  return *reinterpret_cast<const float4 *>(p + e);
+}
+__device__ __forceinline__ void store4(uint16_t *p, long long e, float4 v) {
+  *reinterpret_cast<uint2 *>(p + e) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+}
+__device__ __forceinline__ void store4(float *p, long long e, float4 v) {
+  *reinterpret_cast<float4 *>(p + e) = v;
+}
+
+template <typename T>
+__global__ void pack_kernel(const T *__restrict__ x_txt, int n_txt, const T *__restrict__ x_img,
+                            int n_img, int d, float *__restrict__ resid) {
   const long long nq = static_cast<long long>(n_txt + n_img) * d / 4;
+  const long long txt_elems = static_cast<long long>(n_txt) * d;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < nq;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long e = 4 * i;
-    const long long txt_elems = static_cast<long long>(n_txt) * d;
-    const uint2 v = e < txt_elems ? *reinterpret_cast<const uint2 *>(x_txt + e)
-                                  : *reinterpret_cast<const uint2 *>(x_img + (e - txt_elems));
     reinterpret_cast<float4 *>(resid)[i] =
-        make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
-                    __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+        e < txt_elems ? load4(x_txt, e) : load4(x_img, e - txt_elems);
   }
 }
 
+template <typename T>
 __global__ void unpack_kernel(const float *__restrict__ resid, int n_txt, int n_img, int d,
-                              uint16_t *__restrict__ x_txt, uint16_t *__restrict__ x_img) {
+                              T *__restrict__ x_txt, T *__restrict__ x_img) {
   const long long nq = static_cast<long long>(n_txt + n_img) * d / 4;
+  const long long txt_elems = static_cast<long long>(n_txt) * d;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < nq;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long e = 4 * i;
-    const long long txt_elems = static_cast<long long>(n_txt) * d;
     const float4 v = reinterpret_cast<const float4 *>(resid)[i];
-    const uint2 o = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
     if (e < txt_elems)
-      *reinterpret_cast<uint2 *>(x_txt + e) = o;
+      store4(x_txt, e, v);
     else
-      *reinterpret_cast<uint2 *>(x_img + (e - txt_elems)) = o;
+      store4(x_img, e - txt_elems, v);
   }
 }
 
@@ -303,16 +316,26 @@ cudaError_t launch_rope_table(const GridDesc *grids, int n_grids, int n_txt, int
 }
 
 cudaError_t launch_pack(const void *x_txt, int n_txt, const void *x_img, int n_img, int d,
-                        float *resid, cudaStream_t s) {
-  pack_kernel<<<1184, 256, 0, s>>>(static_cast<const uint16_t *>(x_txt), n_txt,
-                                   static_cast<const uint16_t *>(x_img), n_img, d, resid);
+                        bool fp32_tokens, float *resid, cudaStream_t s) {
+  if (fp32_tokens)
+    pack_kernel<float><<<1184, 256, 0, s>>>(static_cast<const float *>(x_txt), n_txt,
+                                            static_cast<const float *>(x_img), n_img, d, resid);
+  else
+    pack_kernel<uint16_t><<<1184, 256, 0, s>>>(static_cast<const uint16_t *>(x_txt), n_txt,
+                                               static_cast<const uint16_t *>(x_img), n_img, d,
+                                               resid);
   return cudaGetLastError();
 }
 
-cudaError_t launch_unpack(const float *resid, int n_txt, int n_img, int d, void *x_txt,
-                          void *x_img, cudaStream_t s) {
-  unpack_kernel<<<1184, 256, 0, s>>>(resid, n_txt, n_img, d, static_cast<uint16_t *>(x_txt),
-                                     static_cast<uint16_t *>(x_img));
+cudaError_t launch_unpack(const float *resid, int n_txt, int n_img, int d, bool fp32_tokens,
+                          void *x_txt, void *x_img, cudaStream_t s) {
+  if (fp32_tokens)
+    unpack_kernel<float><<<1184, 256, 0, s>>>(resid, n_txt, n_img, d, static_cast<float *>(x_txt),
+                                              static_cast<float *>(x_img));
+  else
+    unpack_kernel<uint16_t><<<1184, 256, 0, s>>>(resid, n_txt, n_img, d,
+                                                 static_cast<uint16_t *>(x_txt),
+                                                 static_cast<uint16_t *>(x_img));
   return cudaGetLastError();
 }
 

@@ -61,8 +61,8 @@ constexpr int kMaxGrids = 32;
 cudaError_t launch_rope_table(const GridDesc *grids, int n_grids, int n_txt, int n,
                               const int sec[3], float theta, float *table, cudaStream_t s);
 cudaError_t launch_pack(const void *x_txt, int n_txt, const void *x_img, int n_img, int d,
-                        float *resid, cudaStream_t s);
-cudaError_t launch_unpack(const float *resid, int n_txt, int n_img, int d, void *x_txt,
-                          void *x_img, cudaStream_t s);
+                        bool fp32_tokens, float *resid, cudaStream_t s);
+cudaError_t launch_unpack(const float *resid, int n_txt, int n_img, int d, bool fp32_tokens,
+                          void *x_txt, void *x_img, cudaStream_t s);
 
 }  // namespace h3

@@ -31,6 +31,9 @@ H3DIT_EPI_GATED_RESIDUAL = 3
 H3DIT_PRECISION_BF16 = 0
 H3DIT_PRECISION_MXFP8 = 1
 
+KERNEL_KINDS = ["time_embed", "adaln", "rmsnorm", "qkv", "attention", "out_proj", "ffn1",
+                "ffn2", "rope_table", "pack"]
+
 
 class h3dit_config(C.Structure):
     _fields_ = [
@@ -38,7 +41,7 @@ class h3dit_config(C.Structure):
         ("ffn", C.c_int32), ("n_blocks", C.c_int32), ("max_tokens", C.c_int32),
         ("rope_sections", C.c_int32 * 3), ("rope_theta", C.c_float),
         ("norm_eps", C.c_float), ("t_scale", C.c_float), ("gelu_tanh", C.c_int32),
-        ("precision", C.c_int32),
+        ("precision", C.c_int32), ("io_fp32", C.c_int32),
     ]
 
 
@@ -84,6 +87,9 @@ def _load() -> C.CDLL:
         "h3dit_rope_table": (i32, [p, C.POINTER(h3dit_grid), i32, i32, p, p]),
         "h3dit_linear": (i32, [p, i32, p, p, i32, i32, i32, p, p, p, p]),
         "h3dit_attention": (i32, [p, p, p, p, i32, p, i32, i32, p]),
+        "h3dit_profile_begin": (i32, [p]),
+        "h3dit_profile_end": (i32, [p, C.POINTER(C.c_float), C.POINTER(C.c_int64)]),
+        "h3dit_launch_count": (C.c_int64, [p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -116,12 +122,13 @@ def check(ctx, status: int) -> None:
 def make_config(hidden: int, heads: int, head_dim: int, ffn: int, n_blocks: int,
                 max_tokens: int, sections: Sequence[int] | None = None,
                 rope_theta: float = 10000.0, norm_eps: float = 1e-6, t_scale: float = 1000.0,
-                gelu_tanh: bool = False, precision: int = H3DIT_PRECISION_BF16) -> h3dit_config:
+                gelu_tanh: bool = False, precision: int = H3DIT_PRECISION_BF16,
+                io_fp32: bool = False) -> h3dit_config:
     if sections is None:
         sections = {96: (16, 16, 16), 128: (16, 24, 24)}.get(head_dim, (0, 0, 0))
     return h3dit_config(hidden, heads, head_dim, ffn, n_blocks, max_tokens,
                         (C.c_int32 * 3)(*sections), rope_theta, norm_eps, t_scale,
-                        int(gelu_tanh), precision)
+                        int(gelu_tanh), precision, int(io_fp32))
 
 
 def grids_array(grids: Sequence[Tuple[int, int, int]]):
@@ -214,6 +221,19 @@ class Context:
         n_txt = 0 if x_txt is None else x_txt.shape[0]
         self._check(lib.h3dit_block_forward(self.handle, block, t, _ptr(mod), _ptr(x_img), g,
                                             len(grids), _ptr(x_txt), n_txt, _stream(stream)))
+
+    def profile_begin(self) -> None:
+        self._check(lib.h3dit_profile_begin(self.handle))
+
+    def profile_end(self) -> dict:
+        """{kind: (total ms, launches)} since profile_begin."""
+        ms = (C.c_float * len(KERNEL_KINDS))()
+        cnt = (C.c_int64 * len(KERNEL_KINDS))()
+        self._check(lib.h3dit_profile_end(self.handle, ms, cnt))
+        return {k: (float(ms[i]), int(cnt[i])) for i, k in enumerate(KERNEL_KINDS)}
+
+    def launch_count(self) -> int:
+        return int(lib.h3dit_launch_count(self.handle))
 
     def step(self, t: float, x_img, grids, x_txt, stream=None) -> None:
         g = grids_array(grids)

@@ -66,6 +66,7 @@ typedef struct h3dit_config {
   float t_scale;            /* sinusoid argument is t_scale * t (1000)                 */
   int32_t gelu_tanh;        /* 0: exact erf GELU, 1: tanh approximation                */
   int32_t precision;        /* H3DIT_PRECISION_BF16 (MXFP8: H3DIT_ERR_UNSUPPORTED)     */
+  int32_t io_fp32;          /* token buffers x_txt / x_img: 0 = bf16, 1 = fp32         */
 } h3dit_config;
 
 /* Timestep MLP, fp32, nn.Linear layout: Linear(256 -> D), SiLU, Linear(D -> D). */
@@ -120,19 +121,22 @@ h3dit_status h3dit_create(const h3dit_config *cfg, const h3dit_time_weights *tim
 void h3dit_destroy(h3dit_ctx *ctx);
 
 /* Run block `block` in place on the packed sequence [x_txt; images]:
- *   x_txt  device bf16 [n_txt, D] (may be NULL when n_txt == 0), in/out;
- *   x_img  device bf16 [sum h*w, D], in/out, images in `grids` order;
+ *   x_txt  device [n_txt, D] (may be NULL when n_txt == 0), in/out;
+ *   x_img  device [sum h*w, D], in/out, images in `grids` order;
+ *          both bf16, or fp32 when cfg->io_fp32 is set;
  *   mod    device fp32 [6, D] modulation for this block, or NULL to compute it
  *          from `t` (timestep MLP then this block's AdaLN projection).
- * The residual stream is kept in fp32 inside the call; the result is rounded
- * to bf16 once. Needs 1 <= n_txt + sum h*w <= max_tokens. */
+ * The residual stream is kept in fp32 inside the call; with bf16 token
+ * buffers the result is rounded to bf16 once. Needs
+ * 1 <= n_txt + sum h*w <= max_tokens. */
 h3dit_status h3dit_block_forward(h3dit_ctx *ctx, int32_t block, float t, const float *mod,
                                  void *x_img, const h3dit_grid *grids, int32_t n_grids,
                                  void *x_txt, int32_t n_txt, void *cuda_stream);
 
 /* One sampling step in place: the timestep MLP and all n_blocks AdaLN
  * projections once, then the n_blocks blocks in order with an fp32 residual
- * stream, rounded to bf16 at the end. Arguments as in h3dit_block_forward. */
+ * stream, written back to the token buffers at the end. Arguments as in
+ * h3dit_block_forward. */
 h3dit_status h3dit_step(h3dit_ctx *ctx, float t, void *x_img, const h3dit_grid *grids,
                         int32_t n_grids, void *x_txt, int32_t n_txt, void *cuda_stream);
 
@@ -183,6 +187,33 @@ h3dit_status h3dit_linear(h3dit_ctx *ctx, int32_t epilogue, const void *a, const
 h3dit_status h3dit_attention(h3dit_ctx *ctx, const void *q, const void *k, const void *v,
                              int32_t ld_qkv, void *o, int32_t ld_o, int32_t n,
                              void *cuda_stream);
+
+/* ---- Measurement hooks (for benchmarks and profilers) ----------------- */
+
+/* Kernel kinds the library launches, for h3dit_profile_end. */
+#define H3DIT_KERNEL_TIME_EMBED 0 /* a1 (two small launches)      */
+#define H3DIT_KERNEL_ADALN 1      /* a2                            */
+#define H3DIT_KERNEL_RMSNORM 2    /* a3, a7                        */
+#define H3DIT_KERNEL_QKV 3        /* a4                            */
+#define H3DIT_KERNEL_ATTENTION 4  /* a5                            */
+#define H3DIT_KERNEL_OUT_PROJ 5   /* a6                            */
+#define H3DIT_KERNEL_FFN1 6       /* a8                            */
+#define H3DIT_KERNEL_FFN2 7       /* a9                            */
+#define H3DIT_KERNEL_ROPE_TABLE 8 /* RoPE table of the sequence    */
+#define H3DIT_KERNEL_PACK 9       /* packing / unpacking tokens    */
+#define H3DIT_KERNEL_COUNT 10
+
+/* Start recording a CUDA event pair around every kernel the context launches
+ * (on the stream it is launched on), dropping earlier records. */
+h3dit_status h3dit_profile_begin(h3dit_ctx *ctx);
+
+/* Stop recording; wait for the recorded events and write, per kernel kind,
+ * the summed device time in ms and the number of launches (arrays of
+ * H3DIT_KERNEL_COUNT entries; either may be NULL). */
+h3dit_status h3dit_profile_end(h3dit_ctx *ctx, float *ms_out, int64_t *launches_out);
+
+/* Kernels this context has enqueued since it was created. */
+int64_t h3dit_launch_count(const h3dit_ctx *ctx);
 
 #ifdef __cplusplus
 }

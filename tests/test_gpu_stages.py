@@ -6,8 +6,8 @@ import pytest
 
 from image_generation_b200 import synth
 from oracle import dit_block as O
-from tests.helpers import (assert_bf16_rounding, assert_close, block_tensors, time_tensors,
-                           to_dev, to_np)
+from tests.helpers import (assert_attention_bound, assert_bf16_rounding, assert_close,
+                           block_tensors, time_tensors, to_dev, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -127,7 +127,7 @@ def test_linear_gated_residual(small, m):
     _ok(ctx)
     ref = x + gate * O.linear(a, w)
     assert_close(to_np(xt), ref, "gated residual", cos_min=0.9999999, rel_max=1e-4)
-    assert_close(to_np(xt) - x, ref - x, "gated residual delta")
+    assert_close((to_np(xt) - x).ravel(), (ref - x).ravel(), "gated residual delta")
 
 
 @pytest.mark.parametrize("which", ["small", "small128"])
@@ -170,7 +170,7 @@ def test_attention(request, which, n, packed):
     ctx.attention(qt, kt, vt, ld, o, I, n)
     _ok(ctx)
     ref = O.attention(q, k, v).reshape(n, I)
-    assert_close(to_np(o), ref, "attention")
+    assert_attention_bound(to_np(o), ref, float(np.abs(v).max()), "attention")
 
 
 def test_attention_identical_keys_give_mean_of_values(small):
