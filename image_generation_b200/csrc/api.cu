@@ -592,6 +592,18 @@ h3dit_status h3dit_step(h3dit_ctx *ctx, float t, void *x_img, const h3dit_grid *
   return run_unpack(ctx, n_txt, n_img, x_txt, x_img, s);
 }
 
+h3dit_status h3dit_time_embed_static(const float *w_t1, const float *b_t1, const float *w_t2,
+                                     const float *b_t2, int32_t hidden, float t, float t_scale,
+                                     float *c_out, void *cuda_stream) {
+  if (!w_t1 || !b_t1 || !w_t2 || !b_t2 || !c_out || !aligned16(w_t2)) return H3DIT_ERR_INVALID_ARG;
+  if (hidden < 1 || hidden % 4) return H3DIT_ERR_INVALID_ARG;
+  if (hidden > H3DIT_STATIC_TIME_MAX_HIDDEN) return H3DIT_ERR_UNSUPPORTED;
+  static_assert(H3DIT_STATIC_TIME_MAX_HIDDEN == kStaticTimeMaxHidden, "scratch size");
+  cudaError_t e = launch_time_embed_static(t, t_scale, w_t1, b_t1, w_t2, b_t2, c_out, hidden,
+                                           static_cast<cudaStream_t>(cuda_stream));
+  return e == cudaSuccess ? H3DIT_OK : H3DIT_ERR_CUDA;
+}
+
 h3dit_status h3dit_profile_begin(h3dit_ctx *ctx) {
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
   ctx->recycle_records();

@@ -7,6 +7,8 @@
 //   packing [text; images] into the fp32 residual and back   pack / unpack
 #include <math.h>
 
+#include <mutex>
+
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -274,6 +276,42 @@ cudaError_t launch_time_embed(float t, float t_scale, const float *w1, const flo
   }
   time_out_kernel<<<grid, 32 * warps, smem, s>>>(w2, b2, hidden, c_out, d);
   return cudaGetLastError();
+}
+
+// Scratch of the allocation-free timestep MLP: the hidden layer between its
+// two GEMVs. Every GPU that loads the library holds these 32 KiB until exit.
+static __device__ __align__(256) float g_time_hidden_scratch[kStaticTimeMaxHidden];
+
+// Device address of the scratch array on the current device, looked up once
+// per device (host code cannot use the symbol itself as a device pointer).
+static cudaError_t time_scratch_address(float **out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static float *addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_time_hidden_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = static_cast<float *>(p);
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_time_embed_static(float t, float t_scale, const float *w1, const float *b1,
+                                     const float *w2, const float *b2, float *c_out, int d,
+                                     cudaStream_t s) {
+  if (d < 1 || d > kStaticTimeMaxHidden) return cudaErrorInvalidValue;
+  float *hidden = nullptr;
+  cudaError_t e = time_scratch_address(&hidden);
+  if (e != cudaSuccess) return e;
+  // the hidden layer is fully rewritten before it is read: nothing to clear
+  return launch_time_embed(t, t_scale, w1, b1, w2, b2, hidden, c_out, d, nullptr, s);
 }
 
 cudaError_t launch_adaln(const float *c, const void *const *w_ada, const float *const *b_ada,

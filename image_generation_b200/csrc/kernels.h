@@ -47,6 +47,12 @@ cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const C
 cudaError_t launch_time_embed(float t, float t_scale, const float *w1, const float *b1,
                               const float *w2, const float *b2, float *hidden, float *c_out,
                               int d, int *status, cudaStream_t s);
+// The timestep MLP with its hidden vector in the library's static scratch
+// array (at most kStaticTimeMaxHidden floats); no allocation.
+constexpr int kStaticTimeMaxHidden = 8192;
+cudaError_t launch_time_embed_static(float t, float t_scale, const float *w1, const float *b1,
+                                     const float *w2, const float *b2, float *c_out, int d,
+                                     cudaStream_t s);
 cudaError_t launch_adaln(const float *c, const void *const *w_ada, const float *const *b_ada,
                          int first, int count, float *mod_out, int d, int num_sms,
                          cudaStream_t s);

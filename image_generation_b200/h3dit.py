@@ -30,6 +30,7 @@ H3DIT_EPI_GATED_RESIDUAL = 3
 
 H3DIT_PRECISION_BF16 = 0
 H3DIT_PRECISION_MXFP8 = 1
+H3DIT_STATIC_TIME_MAX_HIDDEN = 8192
 
 KERNEL_KINDS = ["time_embed", "adaln", "rmsnorm", "qkv", "attention", "out_proj", "ffn1",
                 "ffn2", "rope_table", "pack"]
@@ -87,6 +88,7 @@ def _load() -> C.CDLL:
         "h3dit_rope_table": (i32, [p, C.POINTER(h3dit_grid), i32, i32, p, p]),
         "h3dit_linear": (i32, [p, i32, p, p, i32, i32, i32, p, p, p, p]),
         "h3dit_attention": (i32, [p, p, p, p, i32, p, i32, i32, p]),
+        "h3dit_time_embed_static": (i32, [p, p, p, p, i32, f32, f32, p, p]),
         "h3dit_profile_begin": (i32, [p]),
         "h3dit_profile_end": (i32, [p, C.POINTER(C.c_float), C.POINTER(C.c_int64)]),
         "h3dit_launch_count": (C.c_int64, [p]),

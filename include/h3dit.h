@@ -188,6 +188,38 @@ h3dit_status h3dit_attention(h3dit_ctx *ctx, const void *q, const void *k, const
                              int32_t ld_qkv, void *o, int32_t ld_o, int32_t n,
                              void *cuda_stream);
 
+/* ---- Timestep condition without any device allocation ----------------- */
+
+/* Largest `hidden` h3dit_time_embed_static accepts. */
+#define H3DIT_STATIC_TIME_MAX_HIDDEN 8192
+
+/* a1 without a context or a workspace: c_out = W_t2 SiLU(W_t1 e(t) + b_t1) + b_t2,
+ * the same computation and kernels as h3dit_time_embed. The paper has no
+ * counterpart to this entry point; it exists for callers that cannot allocate
+ * device memory at all - for example code running inside a host application
+ * that owns every device allocation and hands a plugin only the buffers it
+ * reads and writes, or a serving process that forbids allocation after
+ * start-up to keep its footprint fixed. Such a caller cannot provide the
+ * workspace a context needs, so this entry point takes the weights and the
+ * output directly and keeps its one scratch vector (the hidden layer, `hidden`
+ * floats) in a fixed array inside the library.
+ *   w_t1 device fp32 [hidden, 256]; b_t1 [hidden]; w_t2 [hidden, hidden];
+ *   b_t2 [hidden]; c_out device fp32 [hidden]; t_scale as in h3dit_config.
+ * Neither this call nor the library allocates or frees device memory for it.
+ * The scratch array holds H3DIT_STATIC_TIME_MAX_HIDDEN floats (32 KiB) on every
+ * GPU that loads the library, until the process exits; hidden larger than
+ * that returns H3DIT_ERR_UNSUPPORTED, bad pointers or hidden < 1 or not a
+ * multiple of 4 return H3DIT_ERR_INVALID_ARG, both before anything is
+ * enqueued. The first call on a device looks up the array's device address
+ * for that device (once per device, with it current); make that first call
+ * before any stream capture. Every call on a device shares the one array and
+ * overwrites all of it that it reads, so nothing carries over between calls;
+ * two calls that overlap on the GPU (different streams, not ordered) race on
+ * it and must be avoided. */
+h3dit_status h3dit_time_embed_static(const float *w_t1, const float *b_t1, const float *w_t2,
+                                     const float *b_t2, int32_t hidden, float t, float t_scale,
+                                     float *c_out, void *cuda_stream);
+
 /* ---- Measurement hooks (for benchmarks and profilers) ----------------- */
 
 /* Kernel kinds the library launches, for h3dit_profile_end. */
