@@ -2,39 +2,92 @@
 //   O_h = softmax(Q_h K_h^T / sqrt(d_h)) V_h over all tokens, no mask,
 // for the single packed text+image stream.
 //
-// One CTA per (128-query tile, head); the KV sequence is walked in tiles of
-// 128 with an online softmax:
-//   warp 0      TMA: Q once; K and V tiles into a 2-stage ring. Every 128-row
-//               tile is loaded as 64-column boxes (128-byte swizzle) of a 3-D
-//               view [tokens, heads, d_h]; columns past d_h read as zero.
-//   warp 1      MMA: S_j = Q K_j^T (M128 N128, K = d_h) into one of two TMEM
-//               S buffers, then O += P_{j-1} V_{j-1} (M128 N = d_h, K128) with
-//               P from shared memory (K-major) and V as an MN-major operand.
-//   warps 2..5  softmax, one query row per thread: read S_j from TMEM, running
-//               max in log2 units, p = 2^(s*scale*log2e - m), P as bf16 into
-//               shared memory. O is rescaled in TMEM only when the running max
-//               grows by more than 8 (a factor 256); otherwise the stale max is
-//               kept, which leaves the final O / l unchanged.
-// Tensor memory: S0 [0,128), S1 [128,256), O [256, 256 + d_h).
+// One CTA per (256 queries = two 128-row tiles, head). The KV sequence is
+// walked in tiles of 128 with an online softmax, and the two query tiles
+// ping-pong so the tensor core works on one tile while the other's softmax
+// runs:
+//   warp 0      TMA: Q0 and Q1 once; K and V tiles into a 2-stage ring. Every
+//               128-row tile is loaded as 64-column boxes (128-byte swizzle)
+//               of a 3-D view [tokens, heads, d_h]; columns past d_h read 0.
+//   warp 1      MMA, per KV tile j:  PV0_{j-1}, S0_j, PV1_{j-1}, S1_j, with
+//               S_t = Q_t K_j^T (M128 N128 K d_h) into TMEM and
+//               O_t += P_t V_j (M128 N d_h K128) taking P_t from TMEM (the
+//               first 64 columns of S_t, bf16 pairs) and V as an MN-major
+//               operand from shared memory.
+//   warps 2..5  softmax of query tile 0, one row per thread; warps 6..9 the
+//               same for tile 1. Each reads S_t from TMEM, keeps a running
+//               max in log2 units, writes P = 2^(s*scale*log2e - m) back as
+//               bf16 over S_t, and rescales O_t in TMEM only when the running
+//               max grows by more than 8 (a factor 256); otherwise the stale
+//               max is kept, which leaves O / l unchanged. After the last
+//               tile it normalises O_t by the row sum and stores it.
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256, 256+d_h),
+// O1 [384, 384+d_h).
+// Ordering: the MMAs one thread issues run in order, and every S_t commit
+// follows the PV_t that read the previous P_t from the same columns, so when
+// a softmax group sees S_t complete, O_t and the P_t columns are free.
 #include "kernels.h"
 #include "ptx.cuh"
 
 namespace h3 {
 namespace {
 
-constexpr int BQ = 128;
+constexpr int BQ = 128;                      // rows of one query tile
 constexpr int BKV = 128;
-constexpr int NS = 2;                       // K/V ring stages
-constexpr uint32_t BOX = 128 * 128;         // one [128 rows x 64 bf16] swizzled box
-constexpr uint32_t Q_BYTES = 2 * BOX;
-constexpr uint32_t KV_BYTES = 2 * BOX;      // one K or V tile (d_h <= 128)
+constexpr int NS = 2;                        // K/V ring stages
+constexpr uint32_t BOX = 128 * 128;          // one [128 rows x 64 bf16] swizzled box
+constexpr uint32_t Q_BYTES = 2 * BOX;        // one query tile (d_h <= 128)
+constexpr uint32_t KV_BYTES = 2 * BOX;       // one K or V tile
 constexpr uint32_t STAGE_BYTES = 2 * KV_BYTES;
-constexpr uint32_t P_BYTES = 2 * BOX;       // P [128 q x 128 kv] as two 64-kv boxes
-constexpr int THREADS = 192;
-constexpr int NUM_BARS = 1 + 2 * NS + 4 + 2 + 1;
-constexpr int SMEM_BYTES = Q_BYTES + NS * STAGE_BYTES + P_BYTES + 1024 + NUM_BARS * 8 + 16;
+constexpr int THREADS = 320;
+constexpr int NUM_BARS = 1 + 2 * NS + 2 + 2 + 2 + 1;
+constexpr int SMEM_BYTES = 2 * Q_BYTES + NS * STAGE_BYTES + 1024 + NUM_BARS * 8 + 16;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
+constexpr float RESCALE_THRESHOLD = 8.0f;    // log2 units
+
+// Share of the exponentials computed on the FMA pipe instead of the MUFU
+// pipe: 0 none, 1 one pair in four, 2 one pair in two. On paper the MUFU
+// work per KV tile at head_dim 96 (2 x 128 x 128 ex2 at 16 per clock per SM)
+// exceeds the tensor work, but measured on B200 the extra FMA-pipe work costs
+// more than it saves at both head dims, so the default is none.
+#ifdef H3_EXP_EMU
+template <int DH>
+constexpr int kExpEmu = H3_EXP_EMU;
+#else
+template <int DH>
+constexpr int kExpEmu = 0;
+#endif
+
+// 2^x for x <= 126 on the FMA pipe (Cody-Waite split): x = n + f with
+// n = round(x) from the 1.5 * 2^23 rounding trick and |f| <= 1/2; 2^f from a
+// degree-3 polynomial, minimax in relative error on [-1/2, 1/2] (Remez
+// exchange, max relative error 7.5e-5, well below the 2^-9 rounding of bf16
+// P); 2^n is added into the exponent field. Inputs below -126 (masked scores
+// are -inf) clamp to about 2^-126.
+H3_DEV float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float q = fmaf(fmaf(fmaf(0.0551716685f, f, 0.2426111251f), f, 0.6932609677f), f,
+                       0.9999280572f);
+  return __uint_as_float(__float_as_uint(q) + (__float_as_uint(t) << 23));
+}
+
+template <int EMU>
+H3_DEV constexpr bool use_poly(int pair) {
+  return EMU == 1 ? (pair % 4) == 3 : EMU == 2 ? (pair % 2) == 1 : false;
+}
+
+// O_t (+)= P_t V with P_t in TMEM (kind::f16, A from tensor memory).
+H3_DEV void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 template <int DH>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -48,21 +101,18 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const uint32_t sQ = smem_u32(smem);
-  const uint32_t sKV = sQ + Q_BYTES;
-  const uint32_t sP = sKV + NS * STAGE_BYTES;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Q_BYTES + NS * STAGE_BYTES + P_BYTES);
+  const uint32_t sQ = smem_u32(smem);  // Q0 then Q1
+  const uint32_t sKV = sQ + 2 * Q_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 2 * Q_BYTES + NS * STAGE_BYTES);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NUM_BARS);
-  uint8_t *pP = smem + Q_BYTES + NS * STAGE_BYTES;
 
   const uint32_t b0 = smem_u32(bars);
   const uint32_t Q_FULL = b0;
   auto KV_FULL = [&](int s) { return b0 + 8u * (1 + s); };
   auto KV_EMPTY = [&](int s) { return b0 + 8u * (1 + NS + s); };
-  auto S_FULL = [&](int b) { return b0 + 8u * (1 + 2 * NS + b); };
-  auto S_EMPTY = [&](int b) { return b0 + 8u * (3 + 2 * NS + b); };
-  const uint32_t P_FULL = b0 + 8u * (5 + 2 * NS);
-  const uint32_t PV_DONE = b0 + 8u * (6 + 2 * NS);
+  auto S_FULL = [&](int t) { return b0 + 8u * (1 + 2 * NS + t); };
+  auto P_FULL = [&](int t) { return b0 + 8u * (3 + 2 * NS + t); };
+  auto O_FULL = [&](int t) { return b0 + 8u * (5 + 2 * NS + t); };
   const uint32_t DRAIN = b0 + 8u * (7 + 2 * NS);
 
   __shared__ int aborted;
@@ -70,7 +120,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int head = blockIdx.y;
-  const int q0 = blockIdx.x * BQ;
+  const int q0 = blockIdx.x * 2 * BQ;
   const int nkv = p.tiles_kv;
 
   if (threadIdx.x == 0) {
@@ -79,12 +129,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(KV_FULL(s), 1);
       mbar_init(KV_EMPTY(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(S_FULL(b), 1);
-      mbar_init(S_EMPTY(b), 128);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(S_FULL(t), 1);
+      mbar_init(P_FULL(t), 128);
+      mbar_init(O_FULL(t), 1);
     }
-    mbar_init(P_FULL, 128);
-    mbar_init(PV_DONE, 1);
     mbar_init(DRAIN, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tq);
@@ -102,13 +151,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(Q_FULL, DCH * BOX);
-      for (int c = 0; c < DCH; ++c) tma_load_3d(sQ + c * BOX, &tq, 64 * c, head, q0, Q_FULL);
+      mbar_arrive_expect_tx(Q_FULL, 2 * DCH * BOX);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < DCH; ++c)
+          tma_load_3d(sQ + t * Q_BYTES + c * BOX, &tq, 64 * c, head, q0 + t * BQ, Q_FULL);
       int issued = 0;
       for (int j = 0; j < nkv; ++j) {
         const int st = j % NS;
-        const uint32_t ph = (j / NS) & 1;
-        if (!mbar_wait(KV_EMPTY(st), ph ^ 1, p.status)) break;
+        if (!mbar_wait(KV_EMPTY(st), ((j / NS) & 1) ^ 1, p.status)) break;
         mbar_arrive_expect_tx(KV_FULL(st), 2 * DCH * BOX);
         const uint32_t k_dst = sKV + st * STAGE_BYTES;
         const uint32_t v_dst = k_dst + KV_BYTES;
@@ -125,84 +175,98 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t tO = tmem + 256;
-      auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait(P_FULL, i & 1, p.status)) return false;
-        tc_fence_after();
-        const uint32_t v_src = sKV + (i % NS) * STAGE_BYTES + KV_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk) {
-          const uint64_t da = desc_sw128(sP + (kk / 4) * BOX + (kk % 4) * 32, 16, 1024);
-          const uint64_t db = desc_sw128(v_src + kk * 16 * 128, BOX, 1024);
-          umma_bf16(tO, da, db, IDESC_O, (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(KV_EMPTY(i % NS));
-        umma_commit(PV_DONE);
-        return true;
-      };
-      bool ok = mbar_wait(Q_FULL, 0, p.status);
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int st = j % NS;
-        if (!mbar_wait(KV_FULL(st), (j / NS) & 1, p.status)) {
-          ok = false;
-          break;
-        }
-        const int sb = j & 1;
-        if (!mbar_wait(S_EMPTY(sb), ((j >> 1) & 1) ^ 1, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t k_src = sKV + st * STAGE_BYTES;
+      auto issue_s = [&](int t, int j) {
+        const uint32_t k_src = sKV + (j % NS) * STAGE_BYTES;
+        const uint32_t q_src = sQ + t * Q_BYTES;
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t off = (kk / 4) * BOX + (kk % 4) * 32;
-          umma_bf16(tmem + 128 * sb, desc_sw128(sQ + off, 16, 1024),
+          umma_bf16(tmem + 128 * t, desc_sw128(q_src + off, 16, 1024),
                     desc_sw128(k_src + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
         }
-        umma_commit(S_FULL(sb));
-        if (j > 0 && !issue_pv(j - 1)) ok = false;
+        umma_commit(S_FULL(t));
+      };
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t v_src = sKV + (j % NS) * STAGE_BYTES + KV_BYTES;
+        const uint32_t o_tmem = tmem + 256 + 128 * t;
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk) {
+          // A: P_t in TMEM, 16 keys = 8 packed columns per step
+          umma_bf16_ts(o_tmem, tmem + 128 * t + 8 * kk, desc_sw128(v_src + kk * 16 * 128, BOX, 1024),
+                       IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(Q_FULL, 0, p.status) && mbar_wait(KV_FULL(0), 0, p.status);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
       }
-      if (ok) issue_pv(nkv - 1);
+      for (int j = 0; j < nkv && ok; ++j) {
+        const bool more = j + 1 < nkv;
+        // tile 0: PV0_j, then S0_{j+1}
+        if (!mbar_wait(P_FULL(0), j & 1, p.status)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(0, j);
+        if (!more) umma_commit(O_FULL(0));
+        if (more) {
+          if (!mbar_wait(KV_FULL((j + 1) % NS), ((j + 1) / NS) & 1, p.status)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        // tile 1: PV1_j, release K_j / V_j, then S1_{j+1}
+        if (!mbar_wait(P_FULL(1), j & 1, p.status)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(1, j);
+        umma_commit(KV_EMPTY(j % NS));
+        if (!more) umma_commit(O_FULL(1));
+        if (more) issue_s(1, j + 1);
+      }
       umma_commit(DRAIN);
       mbar_wait(DRAIN, 0, p.status, false);
     }
   } else {
-    // softmax warps: warp w reads TMEM lanes [32 (w % 4), +32), one query row each
+    // softmax group t = 0 (warps 2..5) or 1 (warps 6..9); warp w reads TMEM
+    // lanes [32 (w % 4), +32): one query row per thread
+    const int t = (warp - 2) >> 2;
     const int sub = warp & 3;
     const int row = sub * 32 + lane;
-    const uint32_t tl = tmem + (static_cast<uint32_t>(sub * 32) << 16);
+    const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
+    const uint32_t tS = tmem + lane_off + 128 * t;
+    const uint32_t tO = tmem + lane_off + 256 + 128 * t;
     const float sl2 = p.scale_log2;
     float m = 0.f, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      const int sb = j & 1;
-      ok = mbar_wait(S_FULL(sb), (j >> 1) & 1, p.status);
+      ok = mbar_wait(S_FULL(t), j & 1, p.status);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
       float s[BKV];
+      {
+        uint32_t r[BKV];
+        tmem_ld128(tS, r);
 #pragma unroll
-      for (int c = 0; c < BKV / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tl + 128 * sb + 32 * c, r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(r[i]);
+        for (int i = 0; i < BKV; ++i) s[i] = __uint_as_float(r[i]);
       }
-      tc_fence_before();
-      mbar_arrive(S_EMPTY(sb));
-
       const int valid = p.n - j * BKV;
       if (valid < BKV) {
 #pragma unroll
         for (int i = 0; i < BKV; ++i)
           if (i >= valid) s[i] = -INFINITY;
       }
-      float mx = s[0];
+      // row max: eight independent chains of three-input max, then combine
+      float a8[8];
 #pragma unroll
-      for (int i = 1; i < BKV; ++i) mx = fmaxf(mx, s[i]);
+      for (int c = 0; c < 8; ++c) a8[c] = s[c];
+#pragma unroll
+      for (int i = 8; i < BKV; i += 16) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) a8[c] = fmax3(a8[c], s[i + c], s[i + 8 + c]);
+      }
+      float mx = fmax3(fmax3(a8[0], a8[1], a8[2]), fmax3(a8[3], a8[4], a8[5]), fmaxf(a8[6], a8[7]));
       mx *= sl2;
       float alpha = 1.f;
       bool rescale = false;
@@ -213,58 +277,49 @@ __global__ void __launch_bounds__(THREADS, 1)
         m = mx;
         rescale = true;
       }
-      float sum = 0.f;
+      float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       uint32_t pk[BKV / 2];
 #pragma unroll
       for (int i = 0; i < BKV; i += 2) {
-        const float e0 = ex2_approx(fmaf(s[i], sl2, -m));
-        const float e1 = ex2_approx(fmaf(s[i + 1], sl2, -m));
-        sum += e0 + e1;
+        float e0, e1;
+        if (use_poly<kExpEmu<DH>>(i / 2)) {
+          e0 = exp2_poly(fmaf(s[i], sl2, -m));
+          e1 = exp2_poly(fmaf(s[i + 1], sl2, -m));
+        } else {
+          e0 = ex2_approx(fmaf(s[i], sl2, -m));
+          e1 = ex2_approx(fmaf(s[i + 1], sl2, -m));
+        }
+        part[(i / 2) & 7] += e0 + e1;
         pk[i / 2] = pack_bf16x2(e0, e1);
       }
+      const float sum = ((part[0] + part[1]) + (part[2] + part[3])) +
+                        ((part[4] + part[5]) + (part[6] + part[7]));
       l = l * alpha + sum;
-
-      if (j > 0) {
-        // PV(j-1) must be done: it reads the P buffer and accumulates into O.
-        ok = mbar_wait(PV_DONE, (j - 1) & 1, p.status);
-        if (!__all_sync(0xffffffffu, ok)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
+      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+        // PV_t of the previous tile completed before S_t was committed
 #pragma unroll
-          for (int c = 0; c < DH / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tl + 256 + 32 * c, r);
+        for (int c = 0; c < DH / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + 32 * c, r);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(tl + 256 + 32 * c, r);
-          }
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st32(tO + 32 * c, r);
         }
       }
-      // P row into the K-major 128-byte-swizzled layout the MMA reads:
-      // kv chunk q (8 values, 16 bytes) of box q/8 sits at chunk (q%8) ^ (row%8).
-#pragma unroll
-      for (int q = 0; q < BKV / 8; ++q) {
-        uint8_t *dst = pP + (q / 8) * BOX + row * 128 + (((q % 8) ^ (row & 7)) * 16);
-        *reinterpret_cast<uint4 *>(dst) =
-            make_uint4(pk[4 * q + 0], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-      }
-      fence_proxy_async_smem();
+      tmem_st64(tS, pk);
       tc_fence_before();
-      mbar_arrive(P_FULL);
+      mbar_arrive(P_FULL(t));
     }
-    if (ok) ok = mbar_wait(PV_DONE, (nkv - 1) & 1, p.status);
+    if (ok) ok = mbar_wait(O_FULL(t), 0, p.status);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const float inv_l = 1.f / l;
-      const int qrow = q0 + row;
+      const int qrow = q0 + t * BQ + row;
       uint16_t *dst = static_cast<uint16_t *>(p.o) + static_cast<size_t>(qrow) * p.ldo + head * DH;
 #pragma unroll
       for (int c = 0; c < DH / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(tl + 256 + 32 * c, r);
+        tmem_ld32(tO + 32 * c, r);
         if (qrow < p.n) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -301,7 +356,7 @@ cudaError_t launch_dh(const CUtensorMap &q, const CUtensorMap &k, const CUtensor
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  dim3 grid((p.n + BQ - 1) / BQ, heads);
+  dim3 grid((p.n + 2 * BQ - 1) / (2 * BQ), heads);
   attn_fwd_tcgen05<DH><<<grid, THREADS, SMEM_BYTES, s>>>(q, k, v, p);
   return cudaGetLastError();
 }
