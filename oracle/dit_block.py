@@ -292,6 +292,94 @@ def step_forward(x, t: float, tw: Dict[str, np.ndarray], blocks: Sequence[Dict[s
     return x
 
 
+# --- a11: MXFP8 block-scaled linears ("H3-Image Day-0 Support", "Faster DiT":
+# MXFP8 GEMMs for the eligible DiT linears) ------------------------------------
+# The pages name the format only. Reading: the OCP Microscaling (MX) v1.0
+# format - E4M3 elements (bias 7, 3 mantissa bits, no infinities, largest
+# finite 448) sharing one E8M0 scale 2^X per 32 consecutive elements along
+# the reduction axis, X = floor(log2(amax)) - 8 (8 = exponent of E4M3's
+# largest normal); elements rounded to nearest, ties to even, saturating at
+# +-448. All four block linears (QKV, out-projection, FFN1, FFN2) are
+# eligible, for both operands; attention stays bf16.
+
+MX_BLOCK = 32
+E4M3_MAX = 448.0
+
+
+def e4m3_round(v) -> np.ndarray:
+    """Round to the nearest E4M3 value (ties to even), saturating at +-448.
+    Normal values 2^e (1 + m/8), e in [-6, 8]; subnormals m/8 * 2^-6."""
+    v = _f64(v)
+    a = np.abs(v)
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.clip(e, -6, 8)
+    quantum = 2.0 ** (e - 3)
+    q = np.round(a / quantum) * quantum  # numpy rounds half to even
+    q = np.minimum(q, E4M3_MAX)
+    return np.sign(v) * q
+
+
+def mx_scale_exponent(amax) -> np.ndarray:
+    """X = floor(log2(amax)) - 8 per block; blocks of zeros get the smallest
+    E8M0 exponent, -127."""
+    amax = _f64(amax)
+    with np.errstate(divide="ignore"):
+        x = np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - 8
+    return np.where(amax > 0, np.clip(x, -127, 127), -127.0)
+
+
+def mx_quantize(x):
+    """MXFP8 along the last axis (length a multiple of 32): returns the E4M3
+    element values and the per-block scale exponents X (value = q * 2^X)."""
+    x = _f64(x)
+    k = x.shape[-1]
+    if k % MX_BLOCK:
+        raise ValueError("last axis must be a multiple of 32")
+    blocks = x.reshape(x.shape[:-1] + (k // MX_BLOCK, MX_BLOCK))
+    X = mx_scale_exponent(np.max(np.abs(blocks), axis=-1))
+    q = e4m3_round(blocks / 2.0 ** X[..., None])
+    return q.reshape(x.shape), X
+
+
+def mx_dequantize(q, X) -> np.ndarray:
+    q = _f64(q)
+    k = q.shape[-1]
+    blocks = q.reshape(q.shape[:-1] + (k // MX_BLOCK, MX_BLOCK))
+    return (blocks * 2.0 ** _f64(X)[..., None]).reshape(q.shape)
+
+
+def mx_roundtrip(x) -> np.ndarray:
+    return mx_dequantize(*mx_quantize(x))
+
+
+def linear_mx(x, w) -> np.ndarray:
+    """x W^T with both operands MXFP8-quantized along the reduction axis."""
+    return mx_roundtrip(x) @ mx_roundtrip(w).T
+
+
+def block_forward_mx(x, mod, w: Dict[str, np.ndarray], pos: np.ndarray, cfg: BlockConfig,
+                     rows: Optional[Iterable[int]] = None) -> np.ndarray:
+    """block_forward with the four linears on MXFP8 operands (a11)."""
+    x = _f64(x)
+    n = x.shape[0]
+    sh1, sc1, g1, sh2, sc2, g2 = _f64(mod)
+    idx = np.arange(n) if rows is None else np.asarray(list(rows), dtype=np.int64)
+    I = cfg.inner
+    H, d = cfg.heads, cfg.head_dim
+    wqkv = mx_roundtrip(w["w_qkv"])
+    xm = mx_roundtrip(norm_modulate(x, sh1, sc1, cfg.norm_eps))
+    k = apply_rope((xm @ wqkv[I:2 * I].T).reshape(n, H, d), pos, cfg.rope_sections, cfg.rope_theta)
+    v = (xm @ wqkv[2 * I:].T).reshape(n, H, d)
+    q = apply_rope((xm[idx] @ wqkv[:I].T).reshape(len(idx), H, d), pos[idx],
+                   cfg.rope_sections, cfg.rope_theta)
+    o = attention(q, k, v).reshape(len(idx), I)
+    xr = x[idx] + g1 * linear_mx(o, w["w_o"])
+    hm = norm_modulate(xr, sh2, sc2, cfg.norm_eps)
+    u = gelu(linear_mx(hm, w["w_ff1"]), cfg.gelu_tanh)
+    return xr + g2 * linear_mx(u, w["w_ff2"])
+
+
 def block_flops(n: int, hidden: int, inner: int, ffn: int) -> int:
     """Algorithmic flops of one block: QKV 6NDI, out-proj 2NDI, FFN 4NDF,
     attention 4N^2 I (QK^T and PV over all N^2 pairs, no causal halving)."""

@@ -355,3 +355,80 @@ def test_flop_count_matches_linear_shapes():
     I = H * d
     macs = n * D * 3 * I + n * I * D + n * D * Fh + n * Fh * D + H * (n * n * d) * 2
     assert O.block_flops(n, D, I, Fh) == 2 * macs
+
+
+# ---------------------------------------------------------------- MXFP8 (a11)
+
+def _all_e4m3_values():
+    """Every finite E4M3 value, enumerated from the bit fields."""
+    vals = set()
+    for e in range(16):
+        for m in range(8):
+            if e == 15 and m == 7:
+                continue  # the NaN code
+            v = (m / 8.0) * 2.0 ** -6 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7)
+            vals.add(v)
+            vals.add(-v)
+    return np.array(sorted(vals))
+
+
+def test_e4m3_rounding_is_nearest_representable():
+    grid = _all_e4m3_values()
+    assert grid.max() == 448.0 and len(grid) == 253  # 127 positive, 127 negative, one zero
+    assert np.array_equal(O.e4m3_round(grid), grid)  # representable values are fixed
+    g = np.random.default_rng(12)
+    x = np.concatenate([g.normal(size=4000) * 50, g.uniform(-500, 500, 2000), [1e-9, -3e-3]])
+    q = O.e4m3_round(x)
+    assert np.all(np.isin(q, grid))
+    inside = np.abs(x) <= 448
+    # nearest: no representable value is strictly closer
+    dist = np.abs(grid[None, :] - x[inside, None]).min(axis=1)
+    assert np.allclose(np.abs(q[inside] - x[inside]), dist, atol=0)
+    assert np.all(q[~inside] == np.sign(x[~inside]) * 448.0)  # saturation
+    # ties go to the even mantissa: 1 + 1/16 lies between 1 and 1.125
+    assert O.e4m3_round(np.array([1.0625, 1.1875, -1.0625]))[0] == 1.0
+    assert O.e4m3_round(np.array([1.1875]))[0] == 1.25
+    normal = (np.abs(x) >= 2.0 ** -6) & inside
+    assert np.max(np.abs(q[normal] - x[normal]) / np.abs(x[normal])) <= 2.0 ** -4
+
+
+def test_mx_quantize_scales_and_roundtrip():
+    g = np.random.default_rng(13)
+    x = g.normal(size=(5, 96)) * np.array([1e-3, 1.0, 300.0])[np.arange(96) // 32]
+    q, X = O.mx_quantize(x)
+    assert X.shape == (5, 3) and np.array_equal(X, np.floor(X))
+    blocks = np.abs(x).reshape(5, 3, 32).max(axis=2)
+    # the block maximum lands in [256, 512) before rounding, so its code is in [256, 448]
+    assert np.all((blocks / 2.0 ** X >= 256) & (blocks / 2.0 ** X < 512))
+    qmax = np.abs(q).reshape(5, 3, 32).max(axis=2)
+    assert np.all((qmax >= 256) & (qmax <= 448))
+    y = O.mx_dequantize(q, X)
+    big = np.abs(x) >= 2.0 ** (np.repeat(X, 32, axis=1) - 6)
+    assert np.max(np.abs(y - x)[big] / np.abs(x)[big]) <= 2.0 ** -4
+    # values already on the grid survive exactly
+    exact = np.repeat(2.0 ** X, 32, axis=1) * O.e4m3_round(g.uniform(-400, 400, (5, 96)))
+    assert np.array_equal(O.mx_roundtrip(exact), exact)
+    zq, zX = O.mx_quantize(np.zeros((1, 32)))
+    assert np.all(zq == 0) and zX[0, 0] == -127
+
+
+def test_mx_linear_and_block_reduce_to_bf16_block_on_grid_values():
+    """If every operand is already exactly representable in MXFP8, the MXFP8
+    linear equals the plain one."""
+    g = np.random.default_rng(14)
+    x = O.e4m3_round(g.uniform(-300, 300, (7, 64))) * 2.0 ** -5
+    w = O.e4m3_round(g.uniform(-300, 300, (9, 64))) * 2.0 ** -9
+    assert np.allclose(O.linear_mx(x, w), O.linear(x, w), rtol=0, atol=1e-12)
+    cfg = O.config_for(hidden=64, heads=2, head_dim=96, ffn=64)
+    wb = _tiny_weights(cfg, seed=15)
+    pos = O.token_positions(3, [(0, 3, 4)])
+    g2 = np.random.default_rng(16)
+    xb = g2.normal(size=(pos.shape[0], cfg.hidden))
+    mod = g2.normal(size=(6, cfg.hidden)) * 0.3
+    y_mx = O.block_forward_mx(xb, mod, wb, pos, cfg)
+    y = O.block_forward(xb, mod, wb, pos, cfg)
+    d_mx, d = y_mx - xb, y - xb
+    cos = np.sum(d_mx * d) / np.linalg.norm(d_mx) / np.linalg.norm(d)
+    assert 0.99 < cos < 1.0  # close to, but not the same as, the unquantized block
+    mod[2] = mod[5] = 0.0
+    assert np.array_equal(O.block_forward_mx(xb, mod, wb, pos, cfg), xb)
