@@ -47,6 +47,7 @@ def parse():
                     choices=["attention", "qkv", "out_proj", "ffn1", "ffn2", "rmsnorm", "adaln"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-mxfp8", action="store_true")
     return ap.parse_args()
 
 
@@ -159,6 +160,39 @@ def dist_info():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def time_steps(ctx, steps, warmup, x_img, x_txt, grids, barrier, dist):
+    """W warm-up steps, then K steps between barriers; (ms per step, profile,
+    launches), the time being the slowest rank's."""
+    import torch
+
+    ts = timesteps(warmup + steps)
+    for i in range(warmup):
+        ctx.step(ts[i], x_img, grids, x_txt)
+    barrier()
+    if ctx.sync_status() != 0:
+        raise RuntimeError("warm-up failed")
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    ctx.profile_begin()
+    n0 = ctx.launch_count()
+    e0.record(stream)
+    for i in range(steps):
+        ctx.step(ts[warmup + i], x_img, grids, x_txt)
+    e1.record(stream)
+    barrier()
+    launches = ctx.launch_count() - n0
+    prof = ctx.profile_end()
+    elapsed = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([elapsed], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+    if ctx.sync_status() != 0:
+        raise RuntimeError("timed steps failed")
+    return elapsed / steps, prof, launches
 
 
 def make_model(dh: int, seed: int):
@@ -496,6 +530,32 @@ def run_h3dit(args):
             line["cpu_baseline"] = {"value": round(v, 1), "unit": "ms", "cores": threads,
                                     "kind": "oracle", "sample": desc,
                                     "sample_cpu_seconds": round(secs, 1)}
+    # the MXFP8 variant (a11), on the same bf16 weights quantized at create
+    if not args.no_mxfp8:
+        from image_generation_b200 import h3dit as Hb
+
+        cfg_mx = Hb.make_config(D, H, dh, F, L, N_TOK, precision=Hb.H3DIT_PRECISION_MXFP8)
+        ctx_mx = Hb.Context(cfg_mx, tw, blocks)
+        ms_mx, prof_mx, launches_mx = time_steps(ctx_mx, args.steps, args.warmup, x_img, x_txt,
+                                                 grids, barrier, dist)
+        ctx_mx.close()
+        if rank == 0:
+            peaks, peak_src = load_peaks()
+            fp8_peak = 2.0 * float(peaks["bf16_tflops_sustained"])
+            gemm_kinds = ("qkv", "out_proj", "ffn1", "ffn2")
+            gemm_ms = sum(prof_mx[k][0] for k in gemm_kinds)
+            gemm_fl = sum(flops_per_launch(k, N_TOK, dh) * prof_mx[k][1] for k in gemm_kinds)
+            mx = {"ms_per_step": round(ms_mx, 2), "value": round(ms_mx / world, 2), "unit": "ms",
+                  "tflops_step": round(step_flops(N_TOK, dh) / ms_mx / 1e9, 1),
+                  "gemm_tflops": round(gemm_fl / gemm_ms / 1e9, 1),
+                  "gemm_frac_of_fp8_peak": round(gemm_fl / gemm_ms / 1e9 / fp8_peak, 4),
+                  "fp8_peak": fp8_peak,
+                  "fp8_peak_source": f"2 x {peak_src} sustained bf16 (nominal fp8:bf16 = 2)",
+                  "kernels": {k: round(v[0] / max(v[1], 1), 4) for k, v in prof_mx.items() if v[1]},
+                  "gpu_launches": launches_mx}
+            line["mxfp8"] = mx
+            print(json.dumps(line), flush=True)
+    elif rank == 0:
         print(json.dumps(line), flush=True)
     ctx.close()
     if dist is not None:

@@ -21,8 +21,17 @@ namespace {
 constexpr size_t kAlign = 256;
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Per-block MXFP8 weights (E4M3 + scales), made at create.
+struct MxWeights {
+  size_t qkv, qkv_sf, o, o_sf, ff1, ff1_sf, ff2, ff2_sf;
+};
+
 struct Layout {
-  size_t status, resid, xm, qkv, attn, u, mod, cvec, hidden, rope, wptr, bptr, total;
+  size_t status, resid, xm, qkv, attn, u, mod, cvec, hidden, rope, wptr, bptr;
+  // MXFP8 precision only
+  size_t xq, xq_sf, oq, oq_sf, uq, uq_sf, wq, wq_block;
+  MxWeights wq_off;  // offsets inside one block's slice of the wq arena
+  size_t total;
 };
 
 bool config_ok(const h3dit_config *c) {
@@ -38,6 +47,9 @@ bool config_ok(const h3dit_config *c) {
   if (!(c->norm_eps >= 0.f) || !(c->rope_theta > 0.f)) return false;
   if (c->precision != H3DIT_PRECISION_BF16 && c->precision != H3DIT_PRECISION_MXFP8) return false;
   if (c->io_fp32 != 0 && c->io_fp32 != 1) return false;
+  if (c->precision == H3DIT_PRECISION_MXFP8 &&
+      (c->hidden % 128 || (c->heads * c->head_dim) % 128 || c->ffn % 128))
+    return false;
   return true;
 }
 
@@ -63,6 +75,30 @@ Layout plan(const h3dit_config *c) {
   L.rope = take(N * (c->head_dim / 2) * 2 * 4);
   L.wptr = take(static_cast<size_t>(c->n_blocks) * sizeof(void *));
   L.bptr = take(static_cast<size_t>(c->n_blocks) * sizeof(void *));
+  if (c->precision == H3DIT_PRECISION_MXFP8) {
+    L.xq = take(N * D);
+    L.xq_sf = take(mx_sf_bytes(N, D));
+    L.oq = take(N * I);
+    L.oq_sf = take(mx_sf_bytes(N, I));
+    L.uq = take(N * F);
+    L.uq_sf = take(mx_sf_bytes(N, F));
+    size_t b = 0;
+    auto sub = [&](size_t bytes) {
+      const size_t at = b;
+      b = round_up(b + bytes, kAlign);
+      return at;
+    };
+    L.wq_off.qkv = sub(3 * I * D);
+    L.wq_off.qkv_sf = sub(mx_sf_bytes(3 * I, D));
+    L.wq_off.o = sub(D * I);
+    L.wq_off.o_sf = sub(mx_sf_bytes(D, I));
+    L.wq_off.ff1 = sub(F * D);
+    L.wq_off.ff1_sf = sub(mx_sf_bytes(F, D));
+    L.wq_off.ff2 = sub(D * F);
+    L.wq_off.ff2_sf = sub(mx_sf_bytes(D, F));
+    L.wq_block = b;
+    L.wq = take(b * static_cast<size_t>(c->n_blocks));
+  }
   L.total = off;
   return L;
 }
@@ -121,6 +157,8 @@ struct h3dit_ctx {
   const void *const *wptr() { return reinterpret_cast<const void *const *>(ws + L.wptr); }
   const float *const *bptr() { return reinterpret_cast<const float *const *>(ws + L.bptr); }
   int inner() const { return cfg.heads * cfg.head_dim; }
+  bool mx() const { return cfg.precision == H3DIT_PRECISION_MXFP8; }
+  uint8_t *wq(int l, size_t part) { return ws + L.wq + static_cast<size_t>(l) * L.wq_block + part; }
 
   h3dit_status fail(h3dit_status s, const char *fmt, ...) {
     char buf[512];
@@ -274,8 +312,87 @@ h3dit_status run_linear(h3dit_ctx *ctx, int epi, const void *a, const void *w, i
   return ctx->cuda(launch_gemm(ta, tb, p, epi, grid, s), "gemm launch");
 }
 
+h3dit_status encode_fp8(h3dit_ctx *ctx, CUtensorMap *m, const void *base, uint64_t k, uint64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return ctx->fail(H3DIT_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[2] = {k, rows};
+  const cuuint64_t strides[1] = {k};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kGemmMxBK), 128};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return ctx->fail(H3DIT_ERR_CUDA, "tensor map encode failed (%d)", (int)r);
+  return H3DIT_OK;
+}
+
+// MXFP8 linear: a, w E4M3 with scales in the mx layout; epilogues as
+// run_linear, except that GELU writes MXFP8 (out E4M3 [m, n] + out_sf).
+h3dit_status run_linear_mx(h3dit_ctx *ctx, int epi, const void *a, const void *a_sf, const void *w,
+                           const void *w_sf, int m, int n, int k, void *out, long long ldo,
+                           void *out_sf, const float *gate, const float *rope, cudaStream_t s) {
+  if (epi < H3DIT_EPI_STORE || epi > H3DIT_EPI_GATED_RESIDUAL)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "unknown epilogue %d", epi);
+  if (m < 0 || n <= 0 || k <= 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "bad shape %d x %d x %d", m, n, k);
+  if (k % kGemmMxBK || n % kGemmMxBN)
+    return ctx->fail(H3DIT_ERR_UNSUPPORTED, "MXFP8 linear needs k and n multiples of 128 (k=%d n=%d)", k, n);
+  if (!a || !a_sf || !w || !w_sf || !out || !aligned16(a) || !aligned16(a_sf) || !aligned16(w) ||
+      !aligned16(w_sf) || !aligned16(out))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "MXFP8 linear: NULL or misaligned pointer");
+  if (epi == H3DIT_EPI_GATED_RESIDUAL && (!gate || !aligned16(gate)))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "gated residual needs a 16-byte aligned gate");
+  if (epi == H3DIT_EPI_GELU && (!out_sf || ldo != n))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "MXFP8 GELU output needs out_sf and a dense [m, n] out");
+  GemmParams p{};
+  if (epi == H3DIT_EPI_QKV_ROPE) {
+    const int I = ctx->inner(), dh = ctx->cfg.head_dim;
+    const int *sec = ctx->cfg.rope_sections;
+    if (n != 3 * I) return ctx->fail(H3DIT_ERR_INVALID_ARG, "QKV epilogue needs n == 3*heads*head_dim");
+    if (!rope || !aligned16(rope)) return ctx->fail(H3DIT_ERR_INVALID_ARG, "QKV epilogue needs a RoPE table");
+    for (int c = 0; c < 2 * I; c += kGemmMxBN) {
+      const int h = c % dh;
+      if (h != 0 && h != 2 * sec[0] && h != 2 * (sec[0] + sec[1]))
+        return ctx->fail(H3DIT_ERR_UNSUPPORTED, "rope sections do not align with 128-column tiles");
+    }
+    p.head_dim = dh;
+    p.rope_cols = 2 * I;
+    p.sec[0] = sec[0];
+    p.sec[1] = sec[1];
+    p.sec[2] = sec[2];
+  }
+  if (m == 0) return H3DIT_OK;
+  CUtensorMap ta, tb;
+  h3dit_status st = encode_fp8(ctx, &ta, a, k, m);
+  if (st) return st;
+  if ((st = encode_fp8(ctx, &tb, w, k, n))) return st;
+  p.m = m;
+  p.n = n;
+  p.k = k;
+  p.tiles_m = (m + kGemmBM - 1) / kGemmBM;
+  p.tiles_n = n / kGemmMxBN;
+  p.out = out;
+  p.ldo = ldo;
+  p.gate = gate;
+  p.rope = rope;
+  p.gelu_tanh = ctx->cfg.gelu_tanh;
+  p.status = ctx->status();
+  p.a_sf = static_cast<const uint8_t *>(a_sf);
+  p.b_sf = static_cast<const uint8_t *>(w_sf);
+  p.out_sf = static_cast<uint8_t *>(out_sf);
+  const int tiles = p.tiles_m * p.tiles_n;
+  const int grid = tiles < ctx->num_sms ? tiles : ctx->num_sms;
+  const int kernel_epi = epi == H3DIT_EPI_GELU ? kEpiGeluMx : epi;
+  const int kind = epi == H3DIT_EPI_QKV_ROPE   ? H3DIT_KERNEL_QKV
+                   : epi == H3DIT_EPI_GELU     ? H3DIT_KERNEL_FFN1
+                   : k == ctx->inner()         ? H3DIT_KERNEL_OUT_PROJ
+                   : epi == H3DIT_EPI_STORE    ? H3DIT_KERNEL_FFN1
+                                               : H3DIT_KERNEL_FFN2;
+  Launch L(ctx, kind, s);
+  return ctx->cuda(launch_gemm_mx(ta, tb, p, kernel_epi, grid, s), "MXFP8 gemm launch");
+}
+
 h3dit_status run_attention(h3dit_ctx *ctx, const void *q, const void *k, const void *v, int ld,
-                           void *o, int ldo, int n, cudaStream_t s) {
+                           void *o, int ldo, int n, cudaStream_t s, void *o_sf = nullptr) {
   if (n < 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "n < 0");
   if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "attention: NULL or misaligned pointer");
@@ -295,8 +412,11 @@ h3dit_status run_attention(h3dit_ctx *ctx, const void *q, const void *k, const v
   p.ldo = ldo;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(ctx->cfg.head_dim));
   p.status = ctx->status();
+  p.o_sf = static_cast<uint8_t *>(o_sf);
+  if (o_sf && (ldo != I || I % 128 || !aligned16(o_sf)))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "MXFP8 attention output needs ld_o == heads*head_dim, a multiple of 128");
   Launch L(ctx, H3DIT_KERNEL_ATTENTION, s);
-  return ctx->cuda(launch_attention(tq, tk, tv, p, ctx->cfg.head_dim, ctx->cfg.heads, s),
+  return ctx->cuda(launch_attention(tq, tk, tv, p, ctx->cfg.head_dim, ctx->cfg.heads, o_sf != nullptr, s),
                    "attention launch");
 }
 
@@ -333,10 +453,10 @@ h3dit_status rope_table_into(h3dit_ctx *ctx, const h3dit_grid *grids, int n_grid
 }
 
 h3dit_status run_rmsnorm(h3dit_ctx *ctx, const float *x, const float *shift, const float *scale,
-                         void *out, int n, cudaStream_t s) {
+                         void *out, int n, cudaStream_t s, uint8_t *out_sf = nullptr) {
   Launch L(ctx, H3DIT_KERNEL_RMSNORM, s);
   return ctx->cuda(launch_rmsnorm_modulate(x, shift, scale, out, n, ctx->cfg.hidden,
-                                           ctx->cfg.norm_eps, ctx->num_sms, s),
+                                           ctx->cfg.norm_eps, ctx->num_sms, s, out_sf),
                    "rmsnorm launch");
 }
 
@@ -356,8 +476,35 @@ h3dit_status run_unpack(h3dit_ctx *ctx, int n_txt, int n_img, void *x_txt, void 
                    "unpack launch");
 }
 
+// Steps a3..a9 with the four linears on MXFP8 operands (a11).
+h3dit_status block_body_mx(h3dit_ctx *ctx, int l, const float *mod, int n, cudaStream_t s) {
+  const int D = ctx->cfg.hidden, I = ctx->inner(), F = ctx->cfg.ffn;
+  const MxWeights &o = ctx->L.wq_off;
+  uint8_t *xq = ctx->ws + ctx->L.xq, *xq_sf = ctx->ws + ctx->L.xq_sf;
+  uint8_t *oq = ctx->ws + ctx->L.oq, *oq_sf = ctx->ws + ctx->L.oq_sf;
+  uint8_t *uq = ctx->ws + ctx->L.uq, *uq_sf = ctx->ws + ctx->L.uq_sf;
+  h3dit_status st = run_rmsnorm(ctx, ctx->resid(), mod, mod + D, xq, n, s, xq_sf);
+  if (st) return st;
+  if ((st = run_linear_mx(ctx, H3DIT_EPI_QKV_ROPE, xq, xq_sf, ctx->wq(l, o.qkv), ctx->wq(l, o.qkv_sf),
+                          n, 3 * I, D, ctx->qkv(), 3 * I, nullptr, nullptr, ctx->rope(), s)))
+    return st;
+  const uint16_t *qkv = static_cast<const uint16_t *>(ctx->qkv());
+  if ((st = run_attention(ctx, qkv, qkv + I, qkv + 2 * I, 3 * I, oq, I, n, s, oq_sf))) return st;
+  if ((st = run_linear_mx(ctx, H3DIT_EPI_GATED_RESIDUAL, oq, oq_sf, ctx->wq(l, o.o), ctx->wq(l, o.o_sf),
+                          n, D, I, ctx->resid(), D, nullptr, mod + 2 * D, nullptr, s)))
+    return st;
+  if ((st = run_rmsnorm(ctx, ctx->resid(), mod + 3 * D, mod + 4 * D, xq, n, s, xq_sf))) return st;
+  if ((st = run_linear_mx(ctx, H3DIT_EPI_GELU, xq, xq_sf, ctx->wq(l, o.ff1), ctx->wq(l, o.ff1_sf), n,
+                          F, D, uq, F, uq_sf, nullptr, nullptr, s)))
+    return st;
+  return run_linear_mx(ctx, H3DIT_EPI_GATED_RESIDUAL, uq, uq_sf, ctx->wq(l, o.ff2),
+                       ctx->wq(l, o.ff2_sf), n, D, F, ctx->resid(), D, nullptr, mod + 5 * D,
+                       nullptr, s);
+}
+
 // Steps a3..a9 on the packed fp32 residual of n tokens (workspace).
 h3dit_status block_body(h3dit_ctx *ctx, int l, const float *mod, int n, cudaStream_t s) {
+  if (ctx->mx()) return block_body_mx(ctx, l, mod, n, s);
   const h3dit_block_weights &w = ctx->blocks[l];
   const int D = ctx->cfg.hidden, I = ctx->inner(), F = ctx->cfg.ffn;
   const float *sh1 = mod, *sc1 = mod + D, *g1 = mod + 2 * D;
@@ -411,8 +558,16 @@ h3dit_status h3dit_create(const h3dit_config *cfg, const h3dit_time_weights *tim
                           void *cuda_stream, h3dit_ctx **out) {
   if (!out) return H3DIT_ERR_INVALID_ARG;
   *out = nullptr;
-  if (!config_ok(cfg) || !time_w || !blocks) return H3DIT_ERR_INVALID_ARG;
-  if (cfg->precision != H3DIT_PRECISION_BF16) return H3DIT_ERR_UNSUPPORTED;
+  if (!time_w || !blocks) return H3DIT_ERR_INVALID_ARG;
+  if (!config_ok(cfg)) {
+    // a config that is valid but for the MXFP8 shape rules is unsupported, not invalid
+    if (cfg && cfg->precision == H3DIT_PRECISION_MXFP8) {
+      h3dit_config c2 = *cfg;
+      c2.precision = H3DIT_PRECISION_BF16;
+      if (config_ok(&c2)) return H3DIT_ERR_UNSUPPORTED;
+    }
+    return H3DIT_ERR_INVALID_ARG;
+  }
   if (!time_w->w_t1 || !time_w->b_t1 || !time_w->w_t2 || !time_w->b_t2 ||
       !aligned16(time_w->w_t2))
     return H3DIT_ERR_INVALID_ARG;
@@ -454,6 +609,20 @@ h3dit_status h3dit_create(const h3dit_config *cfg, const h3dit_time_weights *tim
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(ctx->ws + L.bptr, bp.data(), bp.size() * sizeof(void *),
                         cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && ctx->mx()) {
+    // MXFP8 copies of the four block linears (a11), quantized once here
+    const int D = cfg->hidden, I = ctx->inner(), F = cfg->ffn;
+    const MxWeights &o = L.wq_off;
+    for (int l = 0; l < cfg->n_blocks && e == cudaSuccess; ++l) {
+      const h3dit_block_weights &b = blocks[l];
+      e = launch_mx_quantize(b.w_qkv, D, 3 * I, D, ctx->wq(l, o.qkv), ctx->wq(l, o.qkv_sf), s);
+      if (e == cudaSuccess) e = launch_mx_quantize(b.w_o, I, D, I, ctx->wq(l, o.o), ctx->wq(l, o.o_sf), s);
+      if (e == cudaSuccess)
+        e = launch_mx_quantize(b.w_ff1, D, F, D, ctx->wq(l, o.ff1), ctx->wq(l, o.ff1_sf), s);
+      if (e == cudaSuccess)
+        e = launch_mx_quantize(b.w_ff2, F, D, F, ctx->wq(l, o.ff2), ctx->wq(l, o.ff2_sf), s);
+    }
+  }
   // the host vectors die with this call: the copies must have been consumed
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
@@ -590,6 +759,56 @@ h3dit_status h3dit_step(h3dit_ctx *ctx, float t, void *x_img, const h3dit_grid *
   for (int l = 0; l < ctx->cfg.n_blocks; ++l)
     if ((st = block_body(ctx, l, ctx->mod(l), n, s))) return st;
   return run_unpack(ctx, n_txt, n_img, x_txt, x_img, s);
+}
+
+size_t h3dit_mx_scale_bytes(int32_t rows, int32_t k) {
+  if (rows <= 0 || k <= 0 || k % 128) return 0;
+  return mx_sf_bytes(rows, k);
+}
+
+h3dit_status h3dit_mx_quantize(h3dit_ctx *ctx, const void *src, int32_t rows, int32_t k, void *dst,
+                               void *sf, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (rows < 0 || k <= 0 || k % 128)
+    return ctx->fail(H3DIT_ERR_UNSUPPORTED, "MXFP8 quantization needs k a multiple of 128");
+  if (!src || !dst || !sf || !aligned16(src) || !aligned16(dst))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "NULL or misaligned pointer");
+  Launch L(ctx, H3DIT_KERNEL_PACK, static_cast<cudaStream_t>(cuda_stream));
+  return ctx->cuda(launch_mx_quantize(src, k, rows, k, static_cast<uint8_t *>(dst),
+                                      static_cast<uint8_t *>(sf),
+                                      static_cast<cudaStream_t>(cuda_stream)),
+                   "quantize launch");
+}
+
+h3dit_status h3dit_linear_mx(h3dit_ctx *ctx, int32_t epilogue, const void *a, const void *a_sf,
+                             const void *w, const void *w_sf, int32_t m, int32_t n, int32_t k,
+                             void *out, void *out_sf, const float *gate, const float *rope_table,
+                             void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  return run_linear_mx(ctx, epilogue, a, a_sf, w, w_sf, m, n, k, out, n, out_sf, gate, rope_table,
+                       static_cast<cudaStream_t>(cuda_stream));
+}
+
+h3dit_status h3dit_rmsnorm_modulate_mx(h3dit_ctx *ctx, const float *x, const float *shift,
+                                       const float *scale, void *out, void *out_sf, int32_t n,
+                                       void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (n < 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "n < 0");
+  if (ctx->cfg.hidden % 128) return ctx->fail(H3DIT_ERR_UNSUPPORTED, "MXFP8 needs hidden % 128 == 0");
+  if (!x || !shift || !scale || !out || !out_sf || !aligned16(x) || !aligned16(shift) ||
+      !aligned16(scale) || !aligned16(out))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "NULL or misaligned pointer");
+  if (n == 0) return H3DIT_OK;
+  return run_rmsnorm(ctx, x, shift, scale, out, n, static_cast<cudaStream_t>(cuda_stream),
+                     static_cast<uint8_t *>(out_sf));
+}
+
+h3dit_status h3dit_attention_mx(h3dit_ctx *ctx, const void *q, const void *k, const void *v,
+                                int32_t ld_qkv, void *o, void *o_sf, int32_t n, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (!o_sf) return ctx->fail(H3DIT_ERR_INVALID_ARG, "o_sf is NULL");
+  return run_attention(ctx, q, k, v, ld_qkv, o, ctx->inner(), n,
+                       static_cast<cudaStream_t>(cuda_stream), o_sf);
 }
 
 h3dit_status h3dit_time_embed_static(const float *w_t1, const float *b_t1, const float *w_t2,

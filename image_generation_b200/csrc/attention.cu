@@ -89,7 +89,9 @@ H3_DEV void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint
       : "memory");
 }
 
-template <int DH>
+// OUT_MX: write O as MXFP8 (E4M3 + a scale per 32 of head_dim) for the
+// MXFP8 out-projection instead of bf16.
+template <int DH, bool OUT_MX>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_fwd_tcgen05(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, const AttnParams p) {
@@ -320,6 +322,22 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int c = 0; c < DH / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(tO + 32 * c, r);
+        if constexpr (OUT_MX) {
+          if (qrow < p.n) {
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * inv_l;
+            uint32_t q[8];
+            const uint32_t sb = mx_quant32(v, q);
+            uint8_t *d8 = static_cast<uint8_t *>(p.o) + static_cast<size_t>(qrow) * p.ldo +
+                          head * DH + 32 * c;
+            st_global_v4(d8, q[0], q[1], q[2], q[3]);
+            st_global_v4(d8 + 16, q[4], q[5], q[6], q[7]);
+            p.o_sf[mx_sf_offset(qrow, (head * DH) / 32 + c, static_cast<int>(p.ldo / 128))] =
+                static_cast<uint8_t>(sb);
+          }
+          continue;
+        }
         if (qrow < p.n) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -346,27 +364,31 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int DH>
+template <int DH, bool OUT_MX>
 cudaError_t launch_dh(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
                       const AttnParams &p, int heads, cudaStream_t s) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tcgen05<DH>,
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tcgen05<DH, OUT_MX>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   dim3 grid((p.n + 2 * BQ - 1) / (2 * BQ), heads);
-  attn_fwd_tcgen05<DH><<<grid, THREADS, SMEM_BYTES, s>>>(q, k, v, p);
+  attn_fwd_tcgen05<DH, OUT_MX><<<grid, THREADS, SMEM_BYTES, s>>>(q, k, v, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
-                             const AttnParams &p, int head_dim, int heads, cudaStream_t s) {
-  if (head_dim == 96) return launch_dh<96>(q, k, v, p, heads, s);
-  if (head_dim == 128) return launch_dh<128>(q, k, v, p, heads, s);
+                             const AttnParams &p, int head_dim, int heads, bool out_mx,
+                             cudaStream_t s) {
+  if (head_dim == 96)
+    return out_mx ? launch_dh<96, true>(q, k, v, p, heads, s) : launch_dh<96, false>(q, k, v, p, heads, s);
+  if (head_dim == 128)
+    return out_mx ? launch_dh<128, true>(q, k, v, p, heads, s)
+                  : launch_dh<128, false>(q, k, v, p, heads, s);
   return cudaErrorInvalidValue;
 }
 

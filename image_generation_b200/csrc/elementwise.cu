@@ -128,10 +128,13 @@ __global__ void __launch_bounds__(kAdaThreads)
 constexpr int kNormThreads = 256;
 constexpr int kNormMaxVec = 8;  // float4s per thread: D <= 8192
 
+// MX: the output is MXFP8 (E4M3 + E8M0 scale per 32), each group of 8
+// consecutive threads holding one 32-element block.
+template <bool MX>
 __global__ void __launch_bounds__(kNormThreads)
     rmsnorm_modulate_kernel(const float *__restrict__ x, const float *__restrict__ shift,
-                            const float *__restrict__ scale, uint16_t *__restrict__ out, int n,
-                            int d, float eps) {
+                            const float *__restrict__ scale, void *__restrict__ out_v,
+                            uint8_t *__restrict__ out_sf, int n, int d, float eps) {
   __shared__ float red[kNormThreads / 32];
   const int nv = d / 4;
   const float inv_d = 1.f / static_cast<float>(d);
@@ -154,18 +157,35 @@ __global__ void __launch_bounds__(kNormThreads)
 #pragma unroll
     for (int w = 0; w < kNormThreads / 32; ++w) tot += red[w];
     const float rinv = rsqrtf(tot * inv_d + eps);
-    uint2 *orow = reinterpret_cast<uint2 *>(out + static_cast<size_t>(row) * d);
 #pragma unroll
     for (int u = 0; u < kNormMaxVec; ++u) {
       const int i = threadIdx.x + u * kNormThreads;
+      if (u * kNormThreads >= nv) break;  // uniform across the block
+      float a = 0.f, b = 0.f, cc = 0.f, dd = 0.f;
       if (i < nv) {
         const float4 sh = __ldg(reinterpret_cast<const float4 *>(shift) + i);
         const float4 sc = __ldg(reinterpret_cast<const float4 *>(scale) + i);
-        const float a = fmaf(v[u].x * rinv, 1.f + sc.x, sh.x);
-        const float b = fmaf(v[u].y * rinv, 1.f + sc.y, sh.y);
-        const float cc = fmaf(v[u].z * rinv, 1.f + sc.z, sh.z);
-        const float dd = fmaf(v[u].w * rinv, 1.f + sc.w, sh.w);
-        orow[i] = make_uint2(pack_bf16x2(a, b), pack_bf16x2(cc, dd));
+        a = fmaf(v[u].x * rinv, 1.f + sc.x, sh.x);
+        b = fmaf(v[u].y * rinv, 1.f + sc.y, sh.y);
+        cc = fmaf(v[u].z * rinv, 1.f + sc.z, sh.z);
+        dd = fmaf(v[u].w * rinv, 1.f + sc.w, sh.w);
+      }
+      if constexpr (MX) {
+        float am = fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(cc), fabsf(dd)));
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
+        const uint32_t sb = mx_scale_byte(am);
+        const float m = mx_inv_scale(sb);
+        if (i < nv) {
+          reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(out_v) +
+                                       static_cast<size_t>(row) * d)[i] =
+              mx_pack4(a * m, b * m, cc * m, dd * m);
+          if ((i & 7) == 0) out_sf[mx_sf_offset(row, i >> 3, d / 128)] = static_cast<uint8_t>(sb);
+        }
+      } else if (i < nv) {
+        reinterpret_cast<uint2 *>(static_cast<uint16_t *>(out_v) + static_cast<size_t>(row) * d)[i] =
+            make_uint2(pack_bf16x2(a, b), pack_bf16x2(cc, dd));
       }
     }
     __syncthreads();  // red[] is reused by the next row
@@ -332,11 +352,15 @@ cudaError_t launch_adaln(const float *c, const void *const *w_ada, const float *
 
 cudaError_t launch_rmsnorm_modulate(const float *x, const float *shift, const float *scale,
                                     void *out, int n, int d, float eps, int num_sms,
-                                    cudaStream_t s) {
+                                    cudaStream_t s, uint8_t *out_sf) {
   if (d > 4 * kNormMaxVec * kNormThreads) return cudaErrorInvalidValue;
   const int grid = n < 8 * num_sms ? n : 8 * num_sms;
-  rmsnorm_modulate_kernel<<<grid, kNormThreads, 0, s>>>(x, shift, scale,
-                                                         static_cast<uint16_t *>(out), n, d, eps);
+  if (out_sf)
+    rmsnorm_modulate_kernel<true><<<grid, kNormThreads, 0, s>>>(x, shift, scale, out, out_sf, n, d,
+                                                                 eps);
+  else
+    rmsnorm_modulate_kernel<false><<<grid, kNormThreads, 0, s>>>(x, shift, scale, out, nullptr, n,
+                                                                  d, eps);
   return cudaGetLastError();
 }
 

@@ -7,7 +7,27 @@
 
 namespace h3 {
 
-enum Epilogue : int { kEpiStore = 0, kEpiQkvRope = 1, kEpiGelu = 2, kEpiGatedResidual = 3 };
+enum Epilogue : int {
+  kEpiStore = 0,
+  kEpiQkvRope = 1,
+  kEpiGelu = 2,
+  kEpiGatedResidual = 3,
+  kEpiGeluMx = 4,  // GELU, written as MXFP8 (E4M3 + per-32 E8M0 scales)
+};
+
+// MXFP8 scale-factor layout (one E8M0 byte per 32 elements along K) for a
+// matrix [rows, K], K a multiple of 128: 512-byte blocks of 128 rows x 4
+// scales, block (row/128, k/128) at ((row/128) * (K/128) + k/128) * 512, and
+// inside a block row r's scale s at (r % 32) * 16 + ((r / 32) % 4) * 4 + s % 4.
+// This is the order tcgen05.cp (32x128b, warpx4) moves into tensor memory
+// for the block-scaled MMA: lane r % 32, column (r / 32) % 4, byte s % 4.
+__host__ __device__ inline size_t mx_sf_offset(int row, int s, int k_chunks) {
+  return (static_cast<size_t>(row >> 7) * k_chunks + (s >> 2)) * 512 + (row & 31) * 16 +
+         ((row >> 5) & 3) * 4 + (s & 3);
+}
+inline size_t mx_sf_bytes(long long rows, long long k) {
+  return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>(k / 128) * 512;
+}
 
 struct GemmParams {
   int m, n, k;
@@ -21,6 +41,9 @@ struct GemmParams {
   int sec[3];             // QKV: rotation pairs per axis
   int gelu_tanh;
   int *status;
+  // MXFP8 only
+  const uint8_t *a_sf, *b_sf;  // scale factors of A [m, k] and W [n, k]
+  uint8_t *out_sf;             // GELU-MXFP8 epilogue: scales of out [m, n]
 };
 
 struct AttnParams {
@@ -30,6 +53,7 @@ struct AttnParams {
   long long ldo;          // elements
   float scale_log2;       // log2(e) / sqrt(head_dim)
   int *status;
+  uint8_t *o_sf;          // MXFP8 output: scales of o [n, heads*head_dim]
 };
 
 // Tile of the tcgen05 GEMM (rows x columns of the output).
@@ -42,7 +66,18 @@ cudaError_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const GemmPa
 int gemm_smem_bytes();
 
 cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
-                             const AttnParams &p, int head_dim, int heads, cudaStream_t s);
+                             const AttnParams &p, int head_dim, int heads, bool out_mx,
+                             cudaStream_t s);
+
+// MXFP8 block-scaled GEMM (tiles 128 x 128, K-blocks of 128): A [m, k] and
+// W [n, k] as E4M3 with scales in the mx_sf layout.
+constexpr int kGemmMxBN = 128;
+constexpr int kGemmMxBK = 128;
+cudaError_t launch_gemm_mx(const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p,
+                           int epilogue, int grid, cudaStream_t s);
+// bf16 [rows, k] (row stride ld elements) -> E4M3 [rows, k] + scales.
+cudaError_t launch_mx_quantize(const void *src, long long ld, int rows, int k, uint8_t *dst,
+                               uint8_t *sf, cudaStream_t s);
 
 cudaError_t launch_time_embed(float t, float t_scale, const float *w1, const float *b1,
                               const float *w2, const float *b2, float *hidden, float *c_out,
@@ -58,7 +93,7 @@ cudaError_t launch_adaln(const float *c, const void *const *w_ada, const float *
                          cudaStream_t s);
 cudaError_t launch_rmsnorm_modulate(const float *x, const float *shift, const float *scale,
                                     void *out, int n, int d, float eps, int num_sms,
-                                    cudaStream_t s);
+                                    cudaStream_t s, uint8_t *out_sf = nullptr);
 
 struct GridDesc {
   int frame, height, width;

@@ -7,6 +7,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -93,6 +94,15 @@ H3_DEV void tma_load_3d(uint32_t dst, const CUtensorMap *m, int x, int y, int z,
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+// Untiled bulk copy global -> shared (16-byte aligned, size a multiple of 16).
+H3_DEV void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
       : "memory");
 }
 
@@ -225,6 +235,71 @@ H3_DEV float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// Shared-memory descriptor of the source of tcgen05.cp 32x128b: 32 rows of
+// 16 bytes, contiguous (no swizzle; 8-row core matrices 128 bytes apart).
+H3_DEV uint64_t desc_sf_copy(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFF) >> 4);
+  d |= static_cast<uint64_t>(1) << 16;    // leading byte offset 16 B (one column; unused)
+  d |= static_cast<uint64_t>(8) << 32;    // stride byte offset 128 B
+  d |= static_cast<uint64_t>(1) << 46;    // version
+  return d;
+}
+// 32 lanes x 128 bits from shared memory into tensor memory, copied to all
+// four lane quarters (the layout block-scaled MMAs read scale factors from).
+H3_DEV void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+// D(tmem) (+)= (A * 2^sfA)(B * 2^sfB), kind::mxf8f6f4 block-scaled, scales in TMEM.
+H3_DEV void umma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                      uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n" ::
+          "r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+// Instruction descriptor, kind::mxf8f6f4 with E4M3 A/B and E8M0 scales:
+// [4,6) B scale byte, [7,10) A format 0 = E4M3, [10,13) B format, [17,23) N >> 3,
+// 23 scale format 1 = E8M0, [24,29) M >> 4, [29,31) A scale byte.
+__host__ __device__ constexpr uint32_t idesc_mxf8(int m, int n, int sf_id) {
+  return (static_cast<uint32_t>(sf_id) << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(m >> 4) << 24) | (static_cast<uint32_t>(sf_id) << 29);
+}
+
+// MXFP8 (OCP MX) quantization of 32 consecutive values: scale exponent
+// X = floor(log2(amax)) - 8 stored as the E8M0 byte X + 127 (0 for a zero or
+// subnormal block), elements v * 2^-X rounded to E4M3 (nearest even,
+// saturating). Returns the scale byte; q holds 32 bytes, element 4i+j in byte
+// j of q[i].
+H3_DEV uint32_t mx_scale_byte(float amax) {
+  const int eb = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF);
+  return eb > 8 ? static_cast<uint32_t>(eb - 8) : 0u;
+}
+H3_DEV float mx_inv_scale(uint32_t sb) { return __uint_as_float((254u - sb) << 23); }  // 2^-X
+H3_DEV uint32_t mx_pack4(float a, float b, float c, float d) {
+  const __nv_fp8x2_storage_t lo =
+      __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const __nv_fp8x2_storage_t hi =
+      __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+H3_DEV uint32_t mx_quant32(const float *v, uint32_t (&q)[8]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t sb = mx_scale_byte(amax);
+  const float mult = mx_inv_scale(sb);
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    q[i] = mx_pack4(v[4 * i] * mult, v[4 * i + 1] * mult, v[4 * i + 2] * mult,
+                    v[4 * i + 3] * mult);
+  return sb;
 }
 
 // ---------------------------------------------------------------- misc

@@ -89,6 +89,11 @@ def _load() -> C.CDLL:
         "h3dit_linear": (i32, [p, i32, p, p, i32, i32, i32, p, p, p, p]),
         "h3dit_attention": (i32, [p, p, p, p, i32, p, i32, i32, p]),
         "h3dit_time_embed_static": (i32, [p, p, p, p, i32, f32, f32, p, p]),
+        "h3dit_mx_scale_bytes": (sz, [i32, i32]),
+        "h3dit_mx_quantize": (i32, [p, p, i32, i32, p, p, p]),
+        "h3dit_linear_mx": (i32, [p, i32, p, p, p, p, i32, i32, i32, p, p, p, p, p]),
+        "h3dit_rmsnorm_modulate_mx": (i32, [p, p, p, p, p, p, i32, p]),
+        "h3dit_attention_mx": (i32, [p, p, p, p, i32, p, p, i32, p]),
         "h3dit_profile_begin": (i32, [p]),
         "h3dit_profile_end": (i32, [p, C.POINTER(C.c_float), C.POINTER(C.c_int64)]),
         "h3dit_launch_count": (C.c_int64, [p]),
@@ -131,6 +136,16 @@ def make_config(hidden: int, heads: int, head_dim: int, ffn: int, n_blocks: int,
     return h3dit_config(hidden, heads, head_dim, ffn, n_blocks, max_tokens,
                         (C.c_int32 * 3)(*sections), rope_theta, norm_eps, t_scale,
                         int(gelu_tanh), precision, int(io_fp32))
+
+
+def mx_scale_bytes(rows: int, k: int) -> int:
+    return int(lib.h3dit_mx_scale_bytes(rows, k))
+
+
+def mx_sf_offset(row: int, s: int, k: int) -> int:
+    """Byte of the scale of row `row`, k-block `s` (32 elements) in the layout
+    the header documents (for decoding in tests)."""
+    return ((row // 128) * (k // 128) + s // 4) * 512 + (row % 32) * 16 + ((row // 32) % 4) * 4 + s % 4
 
 
 def grids_array(grids: Sequence[Tuple[int, int, int]]):
@@ -223,6 +238,28 @@ class Context:
         n_txt = 0 if x_txt is None else x_txt.shape[0]
         self._check(lib.h3dit_block_forward(self.handle, block, t, _ptr(mod), _ptr(x_img), g,
                                             len(grids), _ptr(x_txt), n_txt, _stream(stream)))
+
+    def mx_quantize(self, src, dst, sf, stream=None) -> None:
+        rows, k = src.shape
+        self._check(lib.h3dit_mx_quantize(self.handle, _ptr(src), rows, k, _ptr(dst), _ptr(sf),
+                                          _stream(stream)))
+
+    def linear_mx(self, epilogue: int, a, a_sf, w, w_sf, out, out_sf=None, gate=None,
+                  rope_table=None, stream=None) -> None:
+        m, k = a.shape
+        n = w.shape[0]
+        self._check(lib.h3dit_linear_mx(self.handle, epilogue, _ptr(a), _ptr(a_sf), _ptr(w),
+                                        _ptr(w_sf), m, n, k, _ptr(out), _ptr(out_sf), _ptr(gate),
+                                        _ptr(rope_table), _stream(stream)))
+
+    def rmsnorm_modulate_mx(self, x, shift, scale, out, out_sf, stream=None) -> None:
+        self._check(lib.h3dit_rmsnorm_modulate_mx(self.handle, _ptr(x), _ptr(shift), _ptr(scale),
+                                                  _ptr(out), _ptr(out_sf), x.shape[0],
+                                                  _stream(stream)))
+
+    def attention_mx(self, q, k, v, ld_qkv: int, o, o_sf, n: int, stream=None) -> None:
+        self._check(lib.h3dit_attention_mx(self.handle, _ptr(q), _ptr(k), _ptr(v), ld_qkv,
+                                           _ptr(o), _ptr(o_sf), n, _stream(stream)))
 
     def profile_begin(self) -> None:
         self._check(lib.h3dit_profile_begin(self.handle))

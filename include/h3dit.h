@@ -65,7 +65,9 @@ typedef struct h3dit_config {
   float norm_eps;           /* RMSNorm epsilon (1e-6)                                  */
   float t_scale;            /* sinusoid argument is t_scale * t (1000)                 */
   int32_t gelu_tanh;        /* 0: exact erf GELU, 1: tanh approximation                */
-  int32_t precision;        /* H3DIT_PRECISION_BF16 (MXFP8: H3DIT_ERR_UNSUPPORTED)     */
+  int32_t precision;        /* H3DIT_PRECISION_BF16, or _MXFP8: the four block linears
+                               on MXFP8 operands (hidden, heads*head_dim and ffn must
+                               then be multiples of 128)                            */
   int32_t io_fp32;          /* token buffers x_txt / x_img: 0 = bf16, 1 = fp32         */
 } h3dit_config;
 
@@ -187,6 +189,47 @@ h3dit_status h3dit_linear(h3dit_ctx *ctx, int32_t epilogue, const void *a, const
 h3dit_status h3dit_attention(h3dit_ctx *ctx, const void *q, const void *k, const void *v,
                              int32_t ld_qkv, void *o, int32_t ld_o, int32_t n,
                              void *cuda_stream);
+
+/* ---- a11: the MXFP8 variant of the four block linears ------------------
+ * "H3-Image Day-0 Support: 4K in 0.87s with Vera Rubin", "Faster DiT" and
+ * "Rubin Bringup": MXFP8 GEMMs for the eligible DiT linears. Format (a
+ * reading; the page names it only): OCP MX - E4M3 elements, one E8M0 scale
+ * 2^X per 32 consecutive elements along the reduction axis (K), with
+ * X = floor(log2(amax of the 32)) - 8, elements rounded to nearest even and
+ * saturated at +-448. Scales are stored one byte each (X + 127) in 512-byte
+ * blocks of 128 rows x 4 scales: block (row/128, k/128) at offset
+ * ((row/128) * (K/128) + k/128) * 512, and within it row r's scale for
+ * k-block s at (r % 32) * 16 + ((r / 32) % 4) * 4 + (k/32) % 4.
+ * With cfg->precision = H3DIT_PRECISION_MXFP8, h3dit_create quantizes the
+ * four linears of every block into the workspace, and block_forward / step
+ * run them on MXFP8 activations made by their producers (RMSNorm, the
+ * attention epilogue, the GELU epilogue); attention itself stays bf16. */
+
+/* Bytes of the scale array of a [rows, k] MXFP8 matrix (0 unless k % 128 == 0). */
+size_t h3dit_mx_scale_bytes(int32_t rows, int32_t k);
+
+/* bf16 [rows, k] (device, dense) -> E4M3 [rows, k] (device, one byte each)
+ * plus scales (device, h3dit_mx_scale_bytes(rows, k) bytes). */
+h3dit_status h3dit_mx_quantize(h3dit_ctx *ctx, const void *src, int32_t rows, int32_t k, void *dst,
+                               void *sf, void *cuda_stream);
+
+/* MXFP8 linear: acc = a w^T with a E4M3 [m, k] + a_sf and w E4M3 [n, k] + w_sf;
+ * k and n multiples of 128; epilogues as h3dit_linear, except GELU, which
+ * writes MXFP8: out E4M3 [m, n] + out_sf (h3dit_mx_scale_bytes(m, n)). */
+h3dit_status h3dit_linear_mx(h3dit_ctx *ctx, int32_t epilogue, const void *a, const void *a_sf,
+                             const void *w, const void *w_sf, int32_t m, int32_t n, int32_t k,
+                             void *out, void *out_sf, const float *gate, const float *rope_table,
+                             void *cuda_stream);
+
+/* a3/a7 with an MXFP8 output: out E4M3 [n, D] + out_sf. */
+h3dit_status h3dit_rmsnorm_modulate_mx(h3dit_ctx *ctx, const float *x, const float *shift,
+                                       const float *scale, void *out, void *out_sf, int32_t n,
+                                       void *cuda_stream);
+
+/* a5 with an MXFP8 output for the MXFP8 out-projection: o E4M3
+ * [n, heads*head_dim] (dense) + o_sf; heads*head_dim a multiple of 128. */
+h3dit_status h3dit_attention_mx(h3dit_ctx *ctx, const void *q, const void *k, const void *v,
+                                int32_t ld_qkv, void *o, void *o_sf, int32_t n, void *cuda_stream);
 
 /* ---- Timestep condition without any device allocation ----------------- */
 

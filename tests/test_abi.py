@@ -88,11 +88,14 @@ def test_create_rejects_bad_arguments_before_touching_the_device():
                               C.byref(out)) == H.H3DIT_ERR_INVALID_ARG
     assert H.lib.h3dit_create(C.byref(cfg), C.byref(tw), arr, 0x100000, ws, None, None) \
         == H.H3DIT_ERR_INVALID_ARG
-    # a precision this build does not run
-    mx = _cfg(hidden=768, heads=8, ffn=2048, n_blocks=2, max_tokens=288, precision=1)
+    # MXFP8 with a width that is not a multiple of 128 is not run
+    mx = _cfg(hidden=832, heads=8, ffn=2048, n_blocks=2, max_tokens=288, precision=1)
     tw, arr = _fake_weights(2)
     assert H.lib.h3dit_create(C.byref(mx), C.byref(tw), arr, 0x100000, ws, None,
                               C.byref(out)) == H.H3DIT_ERR_UNSUPPORTED
+    # the MXFP8 workspace also holds the quantized weights
+    mx_ok = _cfg(hidden=768, heads=8, ffn=2048, n_blocks=2, max_tokens=288, precision=1)
+    assert H.lib.h3dit_workspace_bytes(C.byref(mx_ok)) > ws + 2 * (4 * 768 * 768 + 2 * 768 * 2048)
 
 
 def test_null_context_is_rejected_everywhere():
@@ -112,3 +115,14 @@ def test_null_context_is_rejected_everywhere():
         == H.H3DIT_ERR_INVALID_ARG
     H.lib.h3dit_destroy(None)  # NULL-safe
     assert H.lib.h3dit_last_error(None) == b"no context"
+
+
+def test_mx_scale_layout_size():
+    assert H.mx_scale_bytes(128, 128) == 512
+    assert H.mx_scale_bytes(129, 256) == 2 * 2 * 512
+    assert H.mx_scale_bytes(16896, 5376) == 132 * 42 * 512
+    assert H.mx_scale_bytes(100, 96) == 0
+    # every (row, block) of a matrix lands on a distinct byte of the array
+    rows, k = 256, 384
+    offs = {H.mx_sf_offset(r, s, k) for r in range(rows) for s in range(k // 32)}
+    assert len(offs) == rows * k // 32 and max(offs) < H.mx_scale_bytes(rows, k)
