@@ -86,7 +86,8 @@ def load_peaks():
 
 def traffic_for(kind: str, dh: int):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the kernel source as it is now; else None."""
+    the kernel's sources as they are now (every listed file's sha256 must
+    match); else None."""
     path = os.path.join(ROOT, "profiles", f"traffic_{kind}_dh{dh}.txt")
     if not os.path.exists(path):
         return None
@@ -96,12 +97,14 @@ def traffic_for(kind: str, dh: int):
             if ":" in line:
                 k, v = line.split(":", 1)
                 fields[k.strip()] = v.strip()
-    src = fields.get("source")
-    if not src or "sha256" not in fields or "dram_bytes_per_launch" not in fields:
+    srcs = fields.get("sources", "").split()
+    shas = fields.get("sha256", "").split()
+    if not srcs or len(srcs) != len(shas) or "dram_bytes_per_launch" not in fields:
         return None
-    with open(os.path.join(ROOT, src), "rb") as fh:
-        if hashlib.sha256(fh.read()).hexdigest() != fields["sha256"]:
-            return None
+    for src, sha in zip(srcs, shas):
+        with open(os.path.join(ROOT, src), "rb") as fh:
+            if hashlib.sha256(fh.read()).hexdigest() != sha:
+                return None
     return float(fields["dram_bytes_per_launch"])
 
 
@@ -162,6 +165,18 @@ def dist_info():
     return world, rank, local
 
 
+def slowest_rank(value: float, dist, device="cuda") -> float:
+    """The largest of every rank's value (the job is as slow as its slowest
+    replica); identity without a process group."""
+    if dist is None:
+        return value
+    import torch
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def time_steps(ctx, steps, warmup, x_img, x_txt, grids, barrier, dist):
     """W warm-up steps, then K steps between barriers; (ms per step, profile,
     launches), the time being the slowest rank's."""
@@ -185,11 +200,7 @@ def time_steps(ctx, steps, warmup, x_img, x_txt, grids, barrier, dist):
     barrier()
     launches = ctx.launch_count() - n0
     prof = ctx.profile_end()
-    elapsed = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([elapsed], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = slowest_rank(e0.elapsed_time(e1), dist)
     if ctx.sync_status() != 0:
         raise RuntimeError("timed steps failed")
     return elapsed / steps, prof, launches
@@ -431,11 +442,7 @@ def run_h3dit(args):
     launches = ctx.launch_count() - n0
     prof = ctx.profile_end()
     clk = clocks.stop()
-    elapsed = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([elapsed], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = slowest_rank(e0.elapsed_time(e1), dist)
     st = ctx.sync_status()
     if st != 0:
         raise RuntimeError(f"timed steps failed with status {st}")
@@ -465,11 +472,7 @@ def run_h3dit(args):
             e2e_step(ts[i])
         e1.record(stream)
         barrier()
-        e_ms = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([e_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = slowest_rank(e0.elapsed_time(e1), dist)
         nbytes = (h_txt.numel() + h_img.numel()) * h_txt.element_size()
         e2e = {"value": round(e_ms / args.steps / world, 2), "unit": "ms",
                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}

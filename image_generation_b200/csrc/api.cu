@@ -236,16 +236,17 @@ h3dit_status encode_2d(h3dit_ctx *ctx, CUtensorMap *m, const void *base, uint64_
   return H3DIT_OK;
 }
 
-// [tokens, heads, head_dim] view with a token stride of `ld` elements.
+// [tokens, heads, head_dim] view with a token stride of `ld` elements, read
+// in boxes of 64 columns x `box_rows` tokens.
 h3dit_status encode_heads(h3dit_ctx *ctx, CUtensorMap *m, const void *base, int n, int heads,
-                          int head_dim, int ld) {
+                          int head_dim, int ld, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return ctx->fail(H3DIT_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(heads),
                               static_cast<cuuint64_t>(n)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
                                  static_cast<cuuint64_t>(ld) * 2};
-  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -402,12 +403,12 @@ h3dit_status run_attention(h3dit_ctx *ctx, const void *q, const void *k, const v
   if (n == 0) return H3DIT_OK;
   CUtensorMap tq, tk, tv;
   h3dit_status st;
-  if ((st = encode_heads(ctx, &tq, q, n, ctx->cfg.heads, ctx->cfg.head_dim, ld))) return st;
-  if ((st = encode_heads(ctx, &tk, k, n, ctx->cfg.heads, ctx->cfg.head_dim, ld))) return st;
-  if ((st = encode_heads(ctx, &tv, v, n, ctx->cfg.heads, ctx->cfg.head_dim, ld))) return st;
+  if ((st = encode_heads(ctx, &tq, q, n, ctx->cfg.heads, ctx->cfg.head_dim, ld, kAttnBQ))) return st;
+  if ((st = encode_heads(ctx, &tk, k, n, ctx->cfg.heads, ctx->cfg.head_dim, ld, kAttnBKV))) return st;
+  if ((st = encode_heads(ctx, &tv, v, n, ctx->cfg.heads, ctx->cfg.head_dim, ld, kAttnBKV))) return st;
   AttnParams p{};
   p.n = n;
-  p.tiles_kv = (n + 127) / 128;
+  p.tiles_kv = (n + kAttnBKV - 1) / kAttnBKV;
   p.o = o;
   p.ldo = ldo;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(ctx->cfg.head_dim));
@@ -821,6 +822,19 @@ h3dit_status h3dit_time_embed_static(const float *w_t1, const float *b_t1, const
   cudaError_t e = launch_time_embed_static(t, t_scale, w_t1, b_t1, w_t2, b_t2, c_out, hidden,
                                            static_cast<cudaStream_t>(cuda_stream));
   return e == cudaSuccess ? H3DIT_OK : H3DIT_ERR_CUDA;
+}
+
+h3dit_status h3dit_selftest_bounded_wait(h3dit_ctx *ctx, int32_t limit_us, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (limit_us < 1 || limit_us > 1000000)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "limit_us must be in [1, 1e6]");
+  int dev = 0, khz = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev) != cudaSuccess || khz <= 0)
+    khz = 2000000;
+  const long long cycles = static_cast<long long>(limit_us) * (khz / 1000);
+  return ctx->cuda(launch_selftest_wait(ctx->status(), cycles, static_cast<cudaStream_t>(cuda_stream)),
+                   "self-test launch");
 }
 
 h3dit_status h3dit_profile_begin(h3dit_ctx *ctx) {

@@ -3,44 +3,51 @@
 // for the single packed text+image stream.
 //
 // One CTA per (256 queries = two 128-row tiles, head). The KV sequence is
-// walked in tiles of 128 with an online softmax, and the two query tiles
-// ping-pong so the tensor core works on one tile while the other's softmax
-// runs:
-//   warp 0      TMA: Q0 and Q1 once; K and V tiles into a 2-stage ring. Every
-//               128-row tile is loaded as 64-column boxes (128-byte swizzle)
-//               of a 3-D view [tokens, heads, d_h]; columns past d_h read 0.
-//   warp 1      MMA, per KV tile j:  PV0_{j-1}, S0_j, PV1_{j-1}, S1_j, with
-//               S_t = Q_t K_j^T (M128 N128 K d_h) into TMEM and
-//               O_t += P_t V_j (M128 N d_h K128) taking P_t from TMEM (the
-//               first 64 columns of S_t, bf16 pairs) and V as an MN-major
-//               operand from shared memory.
+// walked in tiles of 64 keys with an online softmax. Each query tile owns two
+// S buffers in tensor memory, so the tensor core computes S_t(j+2) while the
+// softmax of tile t works on S_t(j), and the two query tiles interleave:
+//   warp 0      TMA: Q0 and Q1 once; K and V tiles into a 4-stage ring (64-
+//               column boxes of a 3-D [tokens, heads, d_h] view, 128-byte
+//               swizzle; columns past d_h read as zero).
+//   warps 1, 10 MMA issuers, one per query tile t: S_t(j) = Q_t K_j^T (M128
+//               N64 K d_h) into S buffer j % 2 of tile t; O_t += P_t(j) V_j
+//               (M128 N d_h K64) with P_t(j) read from TMEM (the first 32
+//               columns of its S buffer, bf16 pairs) and V as an MN-major
+//               operand from shared memory. Order per j: PV_t(j), S_t(j+2).
+//               One issuer per tile keeps a tile that runs ahead from waiting
+//               behind the other tile's softmax.
 //   warps 2..5  softmax of query tile 0, one row per thread; warps 6..9 the
-//               same for tile 1. Each reads S_t from TMEM, keeps a running
-//               max in log2 units, writes P = 2^(s*scale*log2e - m) back as
-//               bf16 over S_t, and rescales O_t in TMEM only when the running
-//               max grows by more than 8 (a factor 256); otherwise the stale
-//               max is kept, which leaves O / l unchanged. After the last
-//               tile it normalises O_t by the row sum and stores it.
-// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256, 256+d_h),
-// O1 [384, 384+d_h).
-// Ordering: the MMAs one thread issues run in order, and every S_t commit
-// follows the PV_t that read the previous P_t from the same columns, so when
-// a softmax group sees S_t complete, O_t and the P_t columns are free.
+//               same for tile 1: read S_t(j), running max in log2 units,
+//               P = 2^(s*scale*log2e - m) back over S_t(j) as bf16. O_t is
+//               rescaled in TMEM only when the running max grows by more than
+//               8 (a factor 256), after waiting for PV_t(j-1); otherwise the
+//               stale max is kept, which leaves O / l unchanged. After the
+//               last tile it normalises O_t by the row sum and stores it.
+// Tensor memory (512 columns): S buffers of tile t at 64 * (2t + b), b = 0, 1;
+// O0 at [256, 256 + d_h), O1 at [384, 384 + d_h).
+// Ordering: one thread's MMAs run in issue order; S_t(j+2) is issued after
+// PV_t(j), which read P_t(j) from the same columns, by the same thread. A K/V
+// stage is released once both issuers have committed past its last use.
 #include "kernels.h"
 #include "ptx.cuh"
 
 namespace h3 {
 namespace {
 
-constexpr int BQ = 128;                      // rows of one query tile
-constexpr int BKV = 128;
-constexpr int NS = 2;                        // K/V ring stages
-constexpr uint32_t BOX = 128 * 128;          // one [128 rows x 64 bf16] swizzled box
-constexpr uint32_t Q_BYTES = 2 * BOX;        // one query tile (d_h <= 128)
-constexpr uint32_t KV_BYTES = 2 * BOX;       // one K or V tile
+constexpr int BQ = kAttnBQ;                  // rows of one query tile
+constexpr int BKV = kAttnBKV;                // keys per KV tile
+constexpr int NS = 4;                        // K/V ring stages
+constexpr uint32_t QBOX = 128 * 128;         // one [128 rows x 64 bf16] swizzled box
+constexpr uint32_t KBOX = BKV * 128;         // one [64 rows x 64 bf16] swizzled box
+constexpr uint32_t Q_BYTES = 2 * QBOX;       // one query tile (d_h <= 128)
+constexpr uint32_t KV_BYTES = 2 * KBOX;      // one K or V tile
 constexpr uint32_t STAGE_BYTES = 2 * KV_BYTES;
-constexpr int THREADS = 320;
-constexpr int NUM_BARS = 1 + 2 * NS + 2 + 2 + 2 + 1;
+constexpr int THREADS = 352;                 // 11 warps
+// q_full, kv_full/empty[NS], s_full[2][2], p_full[2][2], pv_done[2], o_full[2], drain[2].
+// P_FULL is per S buffer: with two S buffers a softmax group can finish steps
+// j and j+1 before the MMA warp looks for step j, and a single barrier would
+// then have moved two phases, which a parity wait cannot tell apart.
+constexpr int NUM_BARS = 1 + 2 * NS + 4 + 4 + 2 + 2 + 2;
 constexpr int SMEM_BYTES = 2 * Q_BYTES + NS * STAGE_BYTES + 1024 + NUM_BARS * 8 + 16;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;    // log2 units
@@ -58,19 +65,30 @@ template <int DH>
 constexpr int kExpEmu = 0;
 #endif
 
-// 2^x for x <= 126 on the FMA pipe (Cody-Waite split): x = n + f with
-// n = round(x) from the 1.5 * 2^23 rounding trick and |f| <= 1/2; 2^f from a
-// degree-3 polynomial, minimax in relative error on [-1/2, 1/2] (Remez
-// exchange, max relative error 7.5e-5, well below the 2^-9 rounding of bf16
-// P); 2^n is added into the exponent field. Inputs below -126 (masked scores
-// are -inf) clamp to about 2^-126.
-H3_DEV float exp2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float q = fmaf(fmaf(fmaf(0.0551716685f, f, 0.2426111251f), f, 0.6932609677f), f,
-                       0.9999280572f);
-  return __uint_as_float(__float_as_uint(q) + (__float_as_uint(t) << 23));
+// 2^x for x <= 126 on the FMA pipe, two lanes at a time (Cody-Waite
+// split): x = n + f with n = round(x) from the 1.5 * 2^23 rounding trick and
+// |f| <= 1/2; 2^f from a degree-3 polynomial, minimax in relative error on
+// [-1/2, 1/2] (Remez exchange, max relative error 7.5e-5, well below the 2^-9
+// rounding of bf16 P); 2^n is added into the exponent field. Inputs below
+// -126 (masked scores are -inf) clamp to about 2^-126.
+H3_DEV uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  x2 = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t t2 = f2_add(x2, f2_pack(12582912.0f, 12582912.0f));
+  const uint64_t nf2 = f2_add(t2, f2_pack(-12582912.0f, -12582912.0f));  // round(x)
+  float n0, n1;
+  f2_unpack(nf2, n0, n1);
+  const uint64_t f2 = f2_add(x2, f2_pack(-n0, -n1));  // x - round(x)
+  uint64_t q2 = f2_fma(f2_pack(0.0551716685f, 0.0551716685f), f2,
+                       f2_pack(0.2426111251f, 0.2426111251f));
+  q2 = f2_fma(q2, f2, f2_pack(0.6932609677f, 0.6932609677f));
+  q2 = f2_fma(q2, f2, f2_pack(0.9999280572f, 0.9999280572f));
+  float q0, q1, t0, t1;
+  f2_unpack(q2, q0, q1);
+  f2_unpack(t2, t0, t1);
+  return f2_pack(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
 }
 
 template <int EMU>
@@ -90,7 +108,9 @@ H3_DEV void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint
 }
 
 // OUT_MX: write O as MXFP8 (E4M3 + a scale per 32 of head_dim) for the
-// MXFP8 out-projection instead of bf16.
+// MXFP8 out-projection instead of bf16. 352 threads = 11 warps, spread
+// 3/3/3/2 over the four SM sub-partitions, each with a 16K-register file:
+// at most 168 registers per thread.
 template <int DH, bool OUT_MX>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_fwd_tcgen05(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -112,10 +132,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t Q_FULL = b0;
   auto KV_FULL = [&](int s) { return b0 + 8u * (1 + s); };
   auto KV_EMPTY = [&](int s) { return b0 + 8u * (1 + NS + s); };
-  auto S_FULL = [&](int t) { return b0 + 8u * (1 + 2 * NS + t); };
-  auto P_FULL = [&](int t) { return b0 + 8u * (3 + 2 * NS + t); };
-  auto O_FULL = [&](int t) { return b0 + 8u * (5 + 2 * NS + t); };
-  const uint32_t DRAIN = b0 + 8u * (7 + 2 * NS);
+  auto S_FULL = [&](int t, int b) { return b0 + 8u * (1 + 2 * NS + 2 * t + b); };
+  auto P_FULL = [&](int t, int b) { return b0 + 8u * (5 + 2 * NS + 2 * t + b); };
+  auto PV_DONE = [&](int t) { return b0 + 8u * (9 + 2 * NS + t); };
+  auto O_FULL = [&](int t) { return b0 + 8u * (11 + 2 * NS + t); };
+  auto DRAIN = [&](int t) { return b0 + 8u * (13 + 2 * NS + t); };
 
   __shared__ int aborted;
   if (grid_aborted(p.status, &aborted)) return;
@@ -129,14 +150,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(Q_FULL, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(KV_FULL(s), 1);
-      mbar_init(KV_EMPTY(s), 1);
+      mbar_init(KV_EMPTY(s), 2);
     }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(S_FULL(t), 1);
-      mbar_init(P_FULL(t), 128);
+      mbar_init(S_FULL(t, 0), 1);
+      mbar_init(S_FULL(t, 1), 1);
+      mbar_init(P_FULL(t, 0), 128);
+      mbar_init(P_FULL(t, 1), 128);
+      mbar_init(PV_DONE(t), 1);
       mbar_init(O_FULL(t), 1);
     }
-    mbar_init(DRAIN, 1);
+    mbar_init(DRAIN(0), 1);
+    mbar_init(DRAIN(1), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tq);
     tma_prefetch_desc(&tk);
@@ -153,20 +178,20 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(Q_FULL, 2 * DCH * BOX);
+      mbar_arrive_expect_tx(Q_FULL, 2 * DCH * QBOX);
       for (int t = 0; t < 2; ++t)
         for (int c = 0; c < DCH; ++c)
-          tma_load_3d(sQ + t * Q_BYTES + c * BOX, &tq, 64 * c, head, q0 + t * BQ, Q_FULL);
+          tma_load_3d(sQ + t * Q_BYTES + c * QBOX, &tq, 64 * c, head, q0 + t * BQ, Q_FULL);
       int issued = 0;
       for (int j = 0; j < nkv; ++j) {
         const int st = j % NS;
         if (!mbar_wait(KV_EMPTY(st), ((j / NS) & 1) ^ 1, p.status)) break;
-        mbar_arrive_expect_tx(KV_FULL(st), 2 * DCH * BOX);
+        mbar_arrive_expect_tx(KV_FULL(st), 2 * DCH * KBOX);
         const uint32_t k_dst = sKV + st * STAGE_BYTES;
         const uint32_t v_dst = k_dst + KV_BYTES;
         for (int c = 0; c < DCH; ++c) {
-          tma_load_3d(k_dst + c * BOX, &tk, 64 * c, head, j * BKV, KV_FULL(st));
-          tma_load_3d(v_dst + c * BOX, &tv, 64 * c, head, j * BKV, KV_FULL(st));
+          tma_load_3d(k_dst + c * KBOX, &tk, 64 * c, head, j * BKV, KV_FULL(st));
+          tma_load_3d(v_dst + c * KBOX, &tv, 64 * c, head, j * BKV, KV_FULL(st));
         }
         issued = j + 1;
       }
@@ -175,72 +200,67 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int j = issued - 1; j >= 0 && j >= issued - NS; --j)
         mbar_wait(KV_FULL(j % NS), (j / NS) & 1, p.status, false);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 10) {
     if (lane == 0) {
-      auto issue_s = [&](int t, int j) {
+      const int t = warp == 1 ? 0 : 1;
+      const uint32_t s_base = tmem + 128u * t;
+      const uint32_t q_src = sQ + t * Q_BYTES;
+      const uint32_t o_tmem = tmem + 256 + 128 * t;
+      auto issue_s = [&](int j) -> bool {
+        if (!mbar_wait(KV_FULL(j % NS), (j / NS) & 1, p.status)) return false;
+        tc_fence_after();
         const uint32_t k_src = sKV + (j % NS) * STAGE_BYTES;
-        const uint32_t q_src = sQ + t * Q_BYTES;
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
-          const uint32_t off = (kk / 4) * BOX + (kk % 4) * 32;
-          umma_bf16(tmem + 128 * t, desc_sw128(q_src + off, 16, 1024),
-                    desc_sw128(k_src + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+          umma_bf16(s_base + 64u * (j & 1),
+                    desc_sw128(q_src + (kk / 4) * QBOX + (kk % 4) * 32, 16, 1024),
+                    desc_sw128(k_src + (kk / 4) * KBOX + (kk % 4) * 32, 16, 1024), IDESC_S,
+                    kk > 0 ? 1u : 0u);
         }
-        umma_commit(S_FULL(t));
+        umma_commit(S_FULL(t, j & 1));
+        return true;
       };
-      auto issue_pv = [&](int t, int j) {
+      bool ok = mbar_wait(Q_FULL, 0, p.status);
+      for (int j = 0; j < 2 && j < nkv && ok; ++j) ok = issue_s(j);
+      for (int j = 0; j < nkv && ok; ++j) {
+        if (!mbar_wait(P_FULL(t, j & 1), (j >> 1) & 1, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         const uint32_t v_src = sKV + (j % NS) * STAGE_BYTES + KV_BYTES;
-        const uint32_t o_tmem = tmem + 256 + 128 * t;
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk) {
-          // A: P_t in TMEM, 16 keys = 8 packed columns per step
-          umma_bf16_ts(o_tmem, tmem + 128 * t + 8 * kk, desc_sw128(v_src + kk * 16 * 128, BOX, 1024),
-                       IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          // A: P_t(j) in TMEM, 16 keys = 8 packed columns per step
+          umma_bf16_ts(o_tmem, s_base + 64u * (j & 1) + 8 * kk,
+                       desc_sw128(v_src + kk * 16 * 128, KBOX, 1024), IDESC_O,
+                       (j > 0 || kk > 0) ? 1u : 0u);
         }
-      };
-      bool ok = mbar_wait(Q_FULL, 0, p.status) && mbar_wait(KV_FULL(0), 0, p.status);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-      }
-      for (int j = 0; j < nkv && ok; ++j) {
-        const bool more = j + 1 < nkv;
-        // tile 0: PV0_j, then S0_{j+1}
-        if (!mbar_wait(P_FULL(0), j & 1, p.status)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv(0, j);
-        if (!more) umma_commit(O_FULL(0));
-        if (more) {
-          if (!mbar_wait(KV_FULL((j + 1) % NS), ((j + 1) / NS) & 1, p.status)) { ok = false; break; }
-          tc_fence_after();
-          issue_s(0, j + 1);
+        umma_commit(PV_DONE(t));
+        umma_commit(KV_EMPTY(j % NS));  // this tile no longer reads K_j, V_j
+        if (j + 1 == nkv) umma_commit(O_FULL(t));
+        if (j + 2 < nkv && !issue_s(j + 2)) {
+          ok = false;
+          break;
         }
-        // tile 1: PV1_j, release K_j / V_j, then S1_{j+1}
-        if (!mbar_wait(P_FULL(1), j & 1, p.status)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv(1, j);
-        umma_commit(KV_EMPTY(j % NS));
-        if (!more) umma_commit(O_FULL(1));
-        if (more) issue_s(1, j + 1);
       }
-      umma_commit(DRAIN);
-      mbar_wait(DRAIN, 0, p.status, false);
+      umma_commit(DRAIN(t));
+      mbar_wait(DRAIN(t), 0, p.status, false);
     }
   } else {
     // softmax group t = 0 (warps 2..5) or 1 (warps 6..9); warp w reads TMEM
     // lanes [32 (w % 4), +32): one query row per thread
-    const int t = (warp - 2) >> 2;
+    const int t = (warp - 2) >> 2;  // warps 2..9 only: warp 10 is an issuer
     const int sub = warp & 3;
     const int row = sub * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-    const uint32_t tS = tmem + lane_off + 128 * t;
     const uint32_t tO = tmem + lane_off + 256 + 128 * t;
     const float sl2 = p.scale_log2;
     float m = 0.f, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      ok = mbar_wait(S_FULL(t), j & 1, p.status);
+      const uint32_t tS = tmem + lane_off + 64u * (2 * t + (j & 1));
+      ok = mbar_wait(S_FULL(t, j & 1), (j >> 1) & 1, p.status);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
@@ -249,7 +269,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       float s[BKV];
       {
         uint32_t r[BKV];
-        tmem_ld128(tS, r);
+        tmem_ld64(tS, r);
 #pragma unroll
         for (int i = 0; i < BKV; ++i) s[i] = __uint_as_float(r[i]);
       }
@@ -279,26 +299,42 @@ __global__ void __launch_bounds__(THREADS, 1)
         m = mx;
         rescale = true;
       }
-      float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      const uint64_t negm2 = f2_pack(-m, -m);
+      uint64_t part[4] = {0, 0, 0, 0};
       uint32_t pk[BKV / 2];
 #pragma unroll
       for (int i = 0; i < BKV; i += 2) {
-        float e0, e1;
+        const uint64_t y2 = f2_fma(f2_pack(s[i], s[i + 1]), sl2x2, negm2);
+        uint64_t e2;
         if (use_poly<kExpEmu<DH>>(i / 2)) {
-          e0 = exp2_poly(fmaf(s[i], sl2, -m));
-          e1 = exp2_poly(fmaf(s[i + 1], sl2, -m));
+          e2 = exp2_poly2(y2);
         } else {
-          e0 = ex2_approx(fmaf(s[i], sl2, -m));
-          e1 = ex2_approx(fmaf(s[i + 1], sl2, -m));
+          float y0, y1;
+          f2_unpack(y2, y0, y1);
+          e2 = f2_pack(ex2_approx(y0), ex2_approx(y1));
         }
-        part[(i / 2) & 7] += e0 + e1;
+        part[(i / 2) & 3] = f2_add(part[(i / 2) & 3], e2);
+        float e0, e1;
+        f2_unpack(e2, e0, e1);
         pk[i / 2] = pack_bf16x2(e0, e1);
       }
-      const float sum = ((part[0] + part[1]) + (part[2] + part[3])) +
-                        ((part[4] + part[5]) + (part[6] + part[7]));
+      float sum;
+      {
+        const uint64_t t2 = f2_add(f2_add(part[0], part[1]), f2_add(part[2], part[3]));
+        float a0, a1;
+        f2_unpack(t2, a0, a1);
+        sum = a0 + a1;
+      }
       l = l * alpha + sum;
       if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-        // PV_t of the previous tile completed before S_t was committed
+        // O_t must hold PV_t(j-1) in full before it is rescaled
+        ok = mbar_wait(PV_DONE(t), (j - 1) & 1, p.status);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < DH / 32; ++c) {
           uint32_t r[32];
@@ -308,9 +344,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_st32(tO + 32 * c, r);
         }
       }
-      tmem_st64(tS, pk);
+      tmem_st32(tS, pk);
       tc_fence_before();
-      mbar_arrive(P_FULL(t));
+      mbar_arrive(P_FULL(t, j & 1));
     }
     if (ok) ok = mbar_wait(O_FULL(t), 0, p.status);
     if (__all_sync(0xffffffffu, ok)) {

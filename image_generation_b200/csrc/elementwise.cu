@@ -192,6 +192,17 @@ __global__ void __launch_bounds__(kNormThreads)
   }
 }
 
+// ---------------------------------------------------------------- self-test
+__global__ void selftest_wait_kernel(int *status, long long limit_cycles) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+    // nothing ever arrives: the wait must give up and record the timeout
+    mbar_wait_limit(smem_u32(&bar), 0, status, limit_cycles);
+  }
+}
+
 // ---------------------------------------------------------------- RoPE table
 struct GridArray {
   GridDesc g[kMaxGrids];
@@ -361,6 +372,11 @@ cudaError_t launch_rmsnorm_modulate(const float *x, const float *shift, const fl
   else
     rmsnorm_modulate_kernel<false><<<grid, kNormThreads, 0, s>>>(x, shift, scale, out, nullptr, n,
                                                                   d, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_wait(int *status, long long limit_cycles, cudaStream_t s) {
+  selftest_wait_kernel<<<1, 32, 0, s>>>(status, limit_cycles);
   return cudaGetLastError();
 }
 

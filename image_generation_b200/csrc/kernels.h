@@ -65,6 +65,9 @@ cudaError_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const GemmPa
                         int epilogue, int grid, cudaStream_t s);
 int gemm_smem_bytes();
 
+// Attention tiles: 128 queries per query tile (two per CTA), 64 keys per KV tile.
+constexpr int kAttnBQ = 128;
+constexpr int kAttnBKV = 64;
 cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
                              const AttnParams &p, int head_dim, int heads, bool out_mx,
                              cudaStream_t s);
@@ -94,6 +97,10 @@ cudaError_t launch_adaln(const float *c, const void *const *w_ada, const float *
 cudaError_t launch_rmsnorm_modulate(const float *x, const float *shift, const float *scale,
                                     void *out, int n, int d, float eps, int num_sms,
                                     cudaStream_t s, uint8_t *out_sf = nullptr);
+
+// Bounded-wait self-test: one thread waits on an mbarrier that nothing
+// arrives on, gives up after limit_cycles and records the timeout in *status.
+cudaError_t launch_selftest_wait(int *status, long long limit_cycles, cudaStream_t s);
 
 struct GridDesc {
   int frame, height, width;

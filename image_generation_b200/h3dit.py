@@ -94,6 +94,7 @@ def _load() -> C.CDLL:
         "h3dit_linear_mx": (i32, [p, i32, p, p, p, p, i32, i32, i32, p, p, p, p, p]),
         "h3dit_rmsnorm_modulate_mx": (i32, [p, p, p, p, p, p, i32, p]),
         "h3dit_attention_mx": (i32, [p, p, p, p, i32, p, p, i32, p]),
+        "h3dit_selftest_bounded_wait": (i32, [p, i32, p]),
         "h3dit_profile_begin": (i32, [p]),
         "h3dit_profile_end": (i32, [p, C.POINTER(C.c_float), C.POINTER(C.c_int64)]),
         "h3dit_launch_count": (C.c_int64, [p]),
@@ -260,6 +261,9 @@ class Context:
     def attention_mx(self, q, k, v, ld_qkv: int, o, o_sf, n: int, stream=None) -> None:
         self._check(lib.h3dit_attention_mx(self.handle, _ptr(q), _ptr(k), _ptr(v), ld_qkv,
                                            _ptr(o), _ptr(o_sf), n, _stream(stream)))
+
+    def selftest_bounded_wait(self, limit_us: int, stream=None) -> None:
+        self._check(lib.h3dit_selftest_bounded_wait(self.handle, limit_us, _stream(stream)))
 
     def profile_begin(self) -> None:
         self._check(lib.h3dit_profile_begin(self.handle))

@@ -263,6 +263,16 @@ h3dit_status h3dit_time_embed_static(const float *w_t1, const float *b_t1, const
                                      const float *b_t2, int32_t hidden, float t, float t_scale,
                                      float *c_out, void *cuda_stream);
 
+/* ---- Failure detection ---------------------------------------------------
+ * Every wait inside the library's kernels (on an mbarrier fed by TMA or by
+ * another warp) gives up after about one second, records H3DIT_ERR_TIMEOUT in
+ * the context's status word and lets the kernel unwind; kernels that start
+ * while the word is set do no work. h3dit_sync_status reports and clears it.
+ * This entry point exercises that path on purpose without faulting anything:
+ * one thread waits on an mbarrier that nothing arrives on, for limit_us
+ * microseconds (1 .. 1e6), then records the timeout and returns. */
+h3dit_status h3dit_selftest_bounded_wait(h3dit_ctx *ctx, int32_t limit_us, void *cuda_stream);
+
 /* ---- Measurement hooks (for benchmarks and profilers) ----------------- */
 
 /* Kernel kinds the library launches, for h3dit_profile_end. */
