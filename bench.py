@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-mxfp8", action="store_true")
+    ap.add_argument("--mx", action="store_true",
+                    help="with --only qkv/out_proj/ffn1/ffn2: the MXFP8 linear")
     return ap.parse_args()
 
 
@@ -243,7 +245,7 @@ def timesteps(k: int):
 
 # ----------------------------------------------------------------- CPU oracle
 
-def oracle_sample(dh: int, rows_a: int = 8, rows_b: int = 40, seed: int = 0):
+def oracle_sample(dh: int, rows_a: int = 32, rows_b: int = 544, seed: int = 0):
     """Time the oracle on one block of the 4096^2 step for two query-row
     samples (keys and values always over all tokens) and extrapolate linearly
     to all rows and to the 50 blocks of a step, plus the per-step timestep MLP
@@ -354,6 +356,29 @@ def run_only(args):
         qkv = torch.randn(n, 3 * I, device="cuda").bfloat16()
         o = torch.empty(n, I, device="cuda", dtype=torch.bfloat16)
         fn = lambda: ctx.attention(qkv[:, :I], qkv[:, I:2 * I], qkv[:, 2 * I:], 3 * I, o, I, n)
+    elif args.mx and args.only in ("qkv", "ffn1", "out_proj", "ffn2"):
+        w = blk[need]
+        a = torch.randn(n, w.shape[1], device="cuda").bfloat16()
+        aq = torch.empty(n * w.shape[1], dtype=torch.uint8, device="cuda")
+        asf = torch.empty(Hb.mx_scale_bytes(n, w.shape[1]), dtype=torch.uint8, device="cuda")
+        wq = torch.empty(w.numel(), dtype=torch.uint8, device="cuda")
+        wsf = torch.empty(Hb.mx_scale_bytes(w.shape[0], w.shape[1]), dtype=torch.uint8, device="cuda")
+        ctx.mx_quantize(a, aq, asf)
+        ctx.mx_quantize(w, wq, wsf)
+        aq, wq = aq.view(n, -1), wq.view(w.shape[0], -1)
+        if args.only == "qkv":
+            table = torch.empty(n, dh // 2, 2, device="cuda")
+            ctx.rope_table([(0, GRID, GRID)], N_TXT, table)
+            out = torch.empty(n, w.shape[0], device="cuda", dtype=torch.bfloat16)
+            fn = lambda: ctx.linear_mx(Hb.H3DIT_EPI_QKV_ROPE, aq, asf, wq, wsf, out, rope_table=table)
+        elif args.only == "ffn1":
+            out = torch.empty(n * w.shape[0], device="cuda", dtype=torch.uint8)
+            osf = torch.empty(Hb.mx_scale_bytes(n, w.shape[0]), dtype=torch.uint8, device="cuda")
+            fn = lambda: ctx.linear_mx(Hb.H3DIT_EPI_GELU, aq, asf, wq, wsf, out, out_sf=osf)
+        else:
+            x = torch.randn(n, D, device="cuda")
+            gate = torch.full((D,), 0.1, device="cuda")
+            fn = lambda: ctx.linear_mx(Hb.H3DIT_EPI_GATED_RESIDUAL, aq, asf, wq, wsf, x, gate=gate)
     elif args.only in ("qkv", "ffn1"):
         xm = torch.randn(n, D, device="cuda").bfloat16()
         table = torch.empty(n, dh // 2, 2, device="cuda")
@@ -387,7 +412,8 @@ def run_only(args):
     per = ms / max(cnt, 1)
     fl = flops_per_launch(args.only, n, dh)
     by = bytes_per_launch(args.only, n, dh, blocks=1)
-    out = {"kernel": args.only, "head_dim": dh, "tokens": n, "launches": cnt, "ms_per_launch": per}
+    out = {"kernel": args.only + ("_mxfp8" if args.mx else ""), "head_dim": dh, "tokens": n,
+           "launches": cnt, "ms_per_launch": per}
     if fl:
         out["tflops"] = fl / per / 1e9
     if by:

@@ -36,7 +36,8 @@ namespace {
 
 constexpr int BQ = kAttnBQ;                  // rows of one query tile
 constexpr int BKV = kAttnBKV;                // keys per KV tile
-constexpr int NS = 4;                        // K/V ring stages
+constexpr int SBUF = BKV == 64 ? 2 : 1;      // S buffers per query tile (128 columns each tile)
+constexpr int NS = BKV == 64 ? 4 : 2;        // K/V ring stages (128 KiB)
 constexpr uint32_t QBOX = 128 * 128;         // one [128 rows x 64 bf16] swizzled box
 constexpr uint32_t KBOX = BKV * 128;         // one [64 rows x 64 bf16] swizzled box
 constexpr uint32_t Q_BYTES = 2 * QBOX;       // one query tile (d_h <= 128)
@@ -95,6 +96,20 @@ template <int EMU>
 H3_DEV constexpr bool use_poly(int pair) {
   return EMU == 1 ? (pair % 4) == 3 : EMU == 2 ? (pair % 2) == 1 : false;
 }
+
+// TMEM loads / stores of a row's scores (BKV columns) and packed P (BKV/2).
+template <int N>
+H3_DEV void tmem_ld_n(uint32_t taddr, uint32_t (&r)[N]);
+template <>
+H3_DEV void tmem_ld_n<64>(uint32_t taddr, uint32_t (&r)[64]) { tmem_ld64(taddr, r); }
+template <>
+H3_DEV void tmem_ld_n<128>(uint32_t taddr, uint32_t (&r)[128]) { tmem_ld128(taddr, r); }
+template <int N>
+H3_DEV void tmem_st_n(uint32_t taddr, const uint32_t (&r)[N]);
+template <>
+H3_DEV void tmem_st_n<32>(uint32_t taddr, const uint32_t (&r)[32]) { tmem_st32(taddr, r); }
+template <>
+H3_DEV void tmem_st_n<64>(uint32_t taddr, const uint32_t (&r)[64]) { tmem_st64(taddr, r); }
 
 // O_t (+)= P_t V with P_t in TMEM (kind::f16, A from tensor memory).
 H3_DEV void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
@@ -212,18 +227,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t k_src = sKV + (j % NS) * STAGE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
-          umma_bf16(s_base + 64u * (j & 1),
+          umma_bf16(s_base + static_cast<uint32_t>(BKV * (j % SBUF)),
                     desc_sw128(q_src + (kk / 4) * QBOX + (kk % 4) * 32, 16, 1024),
                     desc_sw128(k_src + (kk / 4) * KBOX + (kk % 4) * 32, 16, 1024), IDESC_S,
                     kk > 0 ? 1u : 0u);
         }
-        umma_commit(S_FULL(t, j & 1));
+        umma_commit(S_FULL(t, j % SBUF));
         return true;
       };
       bool ok = mbar_wait(Q_FULL, 0, p.status);
-      for (int j = 0; j < 2 && j < nkv && ok; ++j) ok = issue_s(j);
+      for (int j = 0; j < SBUF && j < nkv && ok; ++j) ok = issue_s(j);
       for (int j = 0; j < nkv && ok; ++j) {
-        if (!mbar_wait(P_FULL(t, j & 1), (j >> 1) & 1, p.status)) {
+        if (!mbar_wait(P_FULL(t, j % SBUF), (j / SBUF) & 1, p.status)) {
           ok = false;
           break;
         }
@@ -232,14 +247,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk) {
           // A: P_t(j) in TMEM, 16 keys = 8 packed columns per step
-          umma_bf16_ts(o_tmem, s_base + 64u * (j & 1) + 8 * kk,
+          umma_bf16_ts(o_tmem, s_base + static_cast<uint32_t>(BKV * (j % SBUF)) + 8 * kk,
                        desc_sw128(v_src + kk * 16 * 128, KBOX, 1024), IDESC_O,
                        (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(PV_DONE(t));
         umma_commit(KV_EMPTY(j % NS));  // this tile no longer reads K_j, V_j
         if (j + 1 == nkv) umma_commit(O_FULL(t));
-        if (j + 2 < nkv && !issue_s(j + 2)) {
+        if (j + SBUF < nkv && !issue_s(j + SBUF)) {
           ok = false;
           break;
         }
@@ -259,8 +274,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     float m = 0.f, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      const uint32_t tS = tmem + lane_off + 64u * (2 * t + (j & 1));
-      ok = mbar_wait(S_FULL(t, j & 1), (j >> 1) & 1, p.status);
+      const uint32_t tS = tmem + lane_off + 128u * t + static_cast<uint32_t>(BKV * (j % SBUF));
+      ok = mbar_wait(S_FULL(t, j % SBUF), (j / SBUF) & 1, p.status);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
@@ -269,7 +284,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       float s[BKV];
       {
         uint32_t r[BKV];
-        tmem_ld64(tS, r);
+        tmem_ld_n<BKV>(tS, r);
 #pragma unroll
         for (int i = 0; i < BKV; ++i) s[i] = __uint_as_float(r[i]);
       }
@@ -344,9 +359,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_st32(tO + 32 * c, r);
         }
       }
-      tmem_st32(tS, pk);
+      tmem_st_n<BKV / 2>(tS, pk);
       tc_fence_before();
-      mbar_arrive(P_FULL(t, j & 1));
+      mbar_arrive(P_FULL(t, j % SBUF));
     }
     if (ok) ok = mbar_wait(O_FULL(t), 0, p.status);
     if (__all_sync(0xffffffffu, ok)) {

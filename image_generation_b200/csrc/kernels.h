@@ -65,9 +65,13 @@ cudaError_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const GemmPa
                         int epilogue, int grid, cudaStream_t s);
 int gemm_smem_bytes();
 
-// Attention tiles: 128 queries per query tile (two per CTA), 64 keys per KV tile.
+// Attention tiles: 128 queries per query tile (two per CTA), kAttnBKV keys per
+// KV tile (64: two S buffers per query tile in TMEM; 128: one).
+#ifndef H3_ATTN_BKV
+#define H3_ATTN_BKV 64
+#endif
 constexpr int kAttnBQ = 128;
-constexpr int kAttnBKV = 64;
+constexpr int kAttnBKV = H3_ATTN_BKV;
 cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
                              const AttnParams &p, int head_dim, int heads, bool out_mx,
                              cudaStream_t s);

@@ -2,10 +2,11 @@
 schedules on the CPU, so that a change to the pipeline cannot deadlock the
 kernel (which would surface on the GPU only as a bounded-wait timeout).
 
-Roles, as in the kernel: a TMA producer over a 4-stage K/V ring; one MMA
-issuer per query tile (S_t(j) into S buffer j % 2, PV_t(j) reading P_t(j),
-S_t(j + 2) issued after PV_t(j)); one softmax group per query tile that may
-wait for PV_t(j - 1) before rescaling O. Barriers complete phases; a wait
+Roles, as in the kernel: a TMA producer over the K/V ring (4 stages with two
+S buffers per query tile, 2 with one); one MMA issuer per query tile (S_t(j)
+into S buffer j % sbuf, PV_t(j) reading P_t(j), S_t(j + sbuf) issued after
+PV_t(j)); one softmax group per query tile that may wait for PV_t(j - 1)
+before rescaling O. Barriers complete phases; a wait
 names a parity and succeeds once the current phase's parity differs, exactly
 the try_wait.parity rule, so a barrier that runs two phases ahead of its
 waiter is a lost wake-up. Each issuer's commits complete in issue order.
@@ -30,18 +31,19 @@ class Barrier:
         return (self.phase & 1) != parity
 
 
-def simulate(nkv, rng, ns=4, p_full_per_buffer=True, rescale_at=()):
+def simulate(nkv, rng, sbuf=2, p_full_per_buffer=True, rescale_at=()):
+    ns = 4 if sbuf == 2 else 2
     bar = Barrier
     q_full = bar("q_full")
     kv_full = [bar(f"kv_full{s}") for s in range(ns)]
     kv_empty = [bar(f"kv_empty{s}", 2) for s in range(ns)]
-    s_full = [[bar(f"s_full{t}{b}") for b in range(2)] for t in range(2)]
+    s_full = [[bar(f"s_full{t}{b}") for b in range(sbuf)] for t in range(2)]
     if p_full_per_buffer:
-        p_full = [[bar(f"p_full{t}{b}") for b in range(2)] for t in range(2)]
-        p_wait = lambda t, j: (p_full[t][j & 1], (j >> 1) & 1)
+        p_full = [[bar(f"p_full{t}{b}") for b in range(sbuf)] for t in range(2)]
+        p_wait = lambda t, j: (p_full[t][j % sbuf], (j // sbuf) & 1)
     else:  # one barrier per tile: the lost-wake-up layout
         one = [bar(f"p_full{t}") for t in range(2)]
-        p_full = [[one[t], one[t]] for t in range(2)]
+        p_full = [[one[t]] * sbuf for t in range(2)]
         p_wait = lambda t, j: (one[t], j & 1)
     pv_done = [bar(f"pv_done{t}") for t in range(2)]
     o_full = [bar(f"o_full{t}") for t in range(2)]
@@ -58,27 +60,27 @@ def simulate(nkv, rng, ns=4, p_full_per_buffer=True, rescale_at=()):
     def issuer(t):
         def issue_s(j):
             yield kv_full[j % ns], (j // ns) & 1
-            pipe[t].append(s_full[t][j & 1])
+            pipe[t].append(s_full[t][j % sbuf])
 
         yield q_full, 0
-        for j in range(min(2, nkv)):
+        for j in range(min(sbuf, nkv)):
             yield from issue_s(j)
         for j in range(nkv):
             yield p_wait(t, j)
             pipe[t].extend([pv_done[t], kv_empty[j % ns]])
             if j + 1 == nkv:
                 pipe[t].append(o_full[t])
-            if j + 2 < nkv:
-                yield from issue_s(j + 2)
+            if j + sbuf < nkv:
+                yield from issue_s(j + sbuf)
         pipe[t].append(drain[t])
         yield drain[t], 0
 
     def softmax(t):
         for j in range(nkv):
-            yield s_full[t][j & 1], (j >> 1) & 1
+            yield s_full[t][j % sbuf], (j // sbuf) & 1
             if j > 0 and (t, j) in rescale_at:
                 yield pv_done[t], (j - 1) & 1
-            p_full[t][j & 1].arrive()
+            p_full[t][j % sbuf].arrive()
         yield o_full[t], 0
 
     roles = {"producer": producer(), "mma0": issuer(0), "mma1": issuer(1),
@@ -110,12 +112,13 @@ def simulate(nkv, rng, ns=4, p_full_per_buffer=True, rescale_at=()):
             if n not in finished and w is not None}
 
 
+@pytest.mark.parametrize("sbuf", [1, 2])
 @pytest.mark.parametrize("nkv", [1, 2, 3, 5, 8, 17, 33])
-def test_attention_pipeline_never_stalls(nkv):
+def test_attention_pipeline_never_stalls(nkv, sbuf):
     rng = random.Random(nkv)
     for _ in range(60):
         rescale = {(t, j) for t in range(2) for j in range(1, nkv) if rng.random() < 0.3}
-        stuck = simulate(nkv, rng, rescale_at=rescale)
+        stuck = simulate(nkv, rng, sbuf=sbuf, rescale_at=rescale)
         assert not stuck, f"stalled with {nkv} KV tiles: {stuck}"
 
 
