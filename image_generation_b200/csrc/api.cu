@@ -286,15 +286,20 @@ h3dit_status run_linear(h3dit_ctx *ctx, int epi, const void *a, const void *w, i
     p.sec[2] = sec[2];
   }
   if (m == 0) return H3DIT_OK;
+  // More than one 128-row block: 256 x 256 tiles on CTA pairs, which halves
+  // the W traffic per SM; a single row block stays on the one-CTA kernel.
+  const int max_pairs = H3_GEMM_PAIR && m > kGemmBM ? gemm_pair_max_clusters(epi) : 0;
+  const bool paired = max_pairs > 0;
   CUtensorMap ta, tb;
   h3dit_status st = encode_2d(ctx, &ta, a, k, m, static_cast<uint64_t>(k) * 2, kGemmBK, kGemmBM);
   if (st) return st;
-  st = encode_2d(ctx, &tb, w, k, n, static_cast<uint64_t>(k) * 2, kGemmBK, kGemmBN);
+  st = encode_2d(ctx, &tb, w, k, n, static_cast<uint64_t>(k) * 2, kGemmBK,
+                 paired ? kGemmBN / 2 : kGemmBN);
   if (st) return st;
   p.m = m;
   p.n = n;
   p.k = k;
-  p.tiles_m = (m + kGemmBM - 1) / kGemmBM;
+  p.tiles_m = (m + (paired ? 2 * kGemmBM : kGemmBM) - 1) / (paired ? 2 * kGemmBM : kGemmBM);
   p.tiles_n = (n + kGemmBN - 1) / kGemmBN;
   p.out = out;
   p.ldo = ldo;
@@ -310,6 +315,11 @@ h3dit_status run_linear(h3dit_ctx *ctx, int epi, const void *a, const void *w, i
                    : epi == H3DIT_EPI_STORE    ? H3DIT_KERNEL_FFN1
                                                : H3DIT_KERNEL_FFN2;
   Launch L(ctx, kind, s);
+  if (paired) {
+    int pairs = tiles < max_pairs ? tiles : max_pairs;
+    if (pairs > ctx->num_sms / 2) pairs = ctx->num_sms / 2;
+    return ctx->cuda(launch_gemm_pair(ta, tb, p, epi, 2 * pairs, s), "paired gemm launch");
+  }
   return ctx->cuda(launch_gemm(ta, tb, p, epi, grid, s), "gemm launch");
 }
 

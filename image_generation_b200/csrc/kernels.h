@@ -65,6 +65,16 @@ cudaError_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const GemmPa
                         int epilogue, int grid, cudaStream_t s);
 int gemm_smem_bytes();
 
+// The same GEMM on 256 x 256 tiles computed by clusters of two CTAs
+// (tcgen05.mma.cta_group::2); grid = 2 x the number of clusters.
+#ifndef H3_GEMM_PAIR
+#define H3_GEMM_PAIR 1
+#endif
+cudaError_t launch_gemm_pair(const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p,
+                             int epilogue, int grid, cudaStream_t s);
+// Clusters of the paired kernel that fit on the device at once (0: unusable).
+int gemm_pair_max_clusters(int epilogue);
+
 // Attention tiles: 128 queries per query tile (two per CTA), kAttnBKV keys per
 // KV tile (64: two S buffers per query tile in TMEM; 128: one).
 #ifndef H3_ATTN_BKV

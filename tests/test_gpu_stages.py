@@ -94,8 +94,8 @@ def _linear_case(m, n, k, seed):
     return a, w
 
 
-@pytest.mark.parametrize("m", [1, 130, 300])
-@pytest.mark.parametrize("n,k", [(768, 768), (2048, 768), (768, 2048)])
+@pytest.mark.parametrize("m", [1, 130, 300, 520])
+@pytest.mark.parametrize("n,k", [(768, 768), (2048, 768), (768, 2048), (800, 768)])
 def test_linear_store_and_gelu(small, m, n, k):
     from image_generation_b200 import h3dit as H
 
@@ -111,6 +111,22 @@ def test_linear_store_and_gelu(small, m, n, k):
     ctx.linear(H.H3DIT_EPI_GELU, to_dev(a), to_dev(w), out)
     _ok(ctx)
     assert_close(to_np(out), O.gelu(ref), "linear+gelu")
+
+
+@pytest.mark.parametrize("k", [64, 192])
+def test_linear_several_tiles_per_cta(small, k):
+    """More output tiles than CTAs: each persistent CTA (or CTA pair) runs
+    several tiles through both TMEM accumulators; a ragged last row block and
+    a short K (one k-block is fewer than the ring's stages)."""
+    from image_generation_b200 import h3dit as H
+
+    ctx, _, _, _ = small
+    m, n = 4500, 4096
+    a, w = _linear_case(m, n, k, 5 + k)
+    out = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+    ctx.linear(H.H3DIT_EPI_STORE, to_dev(a), to_dev(w), out)
+    _ok(ctx)
+    assert_bf16_rounding(to_np(out), O.linear(a, w), "linear", abs_floor=1e-3)
 
 
 @pytest.mark.parametrize("m", [1, 257])
