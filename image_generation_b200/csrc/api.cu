@@ -24,7 +24,10 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Per-block MXFP8 weights (E4M3 + scales), made at create.
 struct MxWeights {
   size_t qkv, qkv_sf, o, o_sf, ff1, ff1_sf, ff2, ff2_sf;
+  // W scales repacked for 224-column tiles (kNoTiled where N is not a multiple of 224)
+  size_t qkv_sft, o_sft, ff1_sft, ff2_sft;
 };
+constexpr size_t kNoTiled = ~static_cast<size_t>(0);
 
 struct Layout {
   size_t status, resid, xm, qkv, attn, u, mod, cvec, hidden, rope, wptr, bptr;
@@ -96,6 +99,13 @@ Layout plan(const h3dit_config *c) {
     L.wq_off.ff1_sf = sub(mx_sf_bytes(F, D));
     L.wq_off.ff2 = sub(D * F);
     L.wq_off.ff2_sf = sub(mx_sf_bytes(D, F));
+    auto tiled = [&](size_t n, size_t k) {
+      return n % kGemmMxWideBN ? kNoTiled : sub(mx_sf_tiled_bytes(n, k));
+    };
+    L.wq_off.qkv_sft = tiled(3 * I, D);
+    L.wq_off.o_sft = tiled(D, I);
+    L.wq_off.ff1_sft = tiled(F, D);
+    L.wq_off.ff2_sft = tiled(D, F);
     L.wq_block = b;
     L.wq = take(b * static_cast<size_t>(c->n_blocks));
   }
@@ -323,12 +333,13 @@ h3dit_status run_linear(h3dit_ctx *ctx, int epi, const void *a, const void *w, i
   return ctx->cuda(launch_gemm(ta, tb, p, epi, grid, s), "gemm launch");
 }
 
-h3dit_status encode_fp8(h3dit_ctx *ctx, CUtensorMap *m, const void *base, uint64_t k, uint64_t rows) {
+h3dit_status encode_fp8(h3dit_ctx *ctx, CUtensorMap *m, const void *base, uint64_t k, uint64_t rows,
+                        uint32_t box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return ctx->fail(H3DIT_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   const cuuint64_t dims[2] = {k, rows};
   const cuuint64_t strides[1] = {k};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kGemmMxBK), 128};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kGemmMxBK), box_rows};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -341,7 +352,8 @@ h3dit_status encode_fp8(h3dit_ctx *ctx, CUtensorMap *m, const void *base, uint64
 // run_linear, except that GELU writes MXFP8 (out E4M3 [m, n] + out_sf).
 h3dit_status run_linear_mx(h3dit_ctx *ctx, int epi, const void *a, const void *a_sf, const void *w,
                            const void *w_sf, int m, int n, int k, void *out, long long ldo,
-                           void *out_sf, const float *gate, const float *rope, cudaStream_t s) {
+                           void *out_sf, const float *gate, const float *rope, cudaStream_t s,
+                           const void *w_sf_tiled = nullptr) {
   if (epi < H3DIT_EPI_STORE || epi > H3DIT_EPI_GATED_RESIDUAL)
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "unknown epilogue %d", epi);
   if (m < 0 || n <= 0 || k <= 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "bad shape %d x %d x %d", m, n, k);
@@ -365,6 +377,11 @@ h3dit_status run_linear_mx(h3dit_ctx *ctx, int epi, const void *a, const void *a
       if (h != 0 && h != 2 * sec[0] && h != 2 * (sec[0] + sec[1]))
         return ctx->fail(H3DIT_ERR_UNSUPPORTED, "rope sections do not align with 128-column tiles");
     }
+    // wide tiles only where each 224-column tile starts on a section boundary
+    for (int c = 0; c < 2 * I && w_sf_tiled; c += kGemmMxWideBN) {
+      const int h = c % dh;
+      if (h != 0 && h != 2 * sec[0] && h != 2 * (sec[0] + sec[1])) w_sf_tiled = nullptr;
+    }
     p.head_dim = dh;
     p.rope_cols = 2 * I;
     p.sec[0] = sec[0];
@@ -372,15 +389,17 @@ h3dit_status run_linear_mx(h3dit_ctx *ctx, int epi, const void *a, const void *a
     p.sec[2] = sec[2];
   }
   if (m == 0) return H3DIT_OK;
+  const bool wide = w_sf_tiled && n % kGemmMxWideBN == 0;
+  const int bn = wide ? kGemmMxWideBN : kGemmMxBN;
   CUtensorMap ta, tb;
   h3dit_status st = encode_fp8(ctx, &ta, a, k, m);
   if (st) return st;
-  if ((st = encode_fp8(ctx, &tb, w, k, n))) return st;
+  if ((st = encode_fp8(ctx, &tb, w, k, n, bn))) return st;
   p.m = m;
   p.n = n;
   p.k = k;
   p.tiles_m = (m + kGemmBM - 1) / kGemmBM;
-  p.tiles_n = n / kGemmMxBN;
+  p.tiles_n = n / bn;
   p.out = out;
   p.ldo = ldo;
   p.gate = gate;
@@ -388,7 +407,7 @@ h3dit_status run_linear_mx(h3dit_ctx *ctx, int epi, const void *a, const void *a
   p.gelu_tanh = ctx->cfg.gelu_tanh;
   p.status = ctx->status();
   p.a_sf = static_cast<const uint8_t *>(a_sf);
-  p.b_sf = static_cast<const uint8_t *>(w_sf);
+  p.b_sf = static_cast<const uint8_t *>(wide ? w_sf_tiled : w_sf);
   p.out_sf = static_cast<uint8_t *>(out_sf);
   const int tiles = p.tiles_m * p.tiles_n;
   const int grid = tiles < ctx->num_sms ? tiles : ctx->num_sms;
@@ -399,7 +418,7 @@ h3dit_status run_linear_mx(h3dit_ctx *ctx, int epi, const void *a, const void *a
                    : epi == H3DIT_EPI_STORE    ? H3DIT_KERNEL_FFN1
                                                : H3DIT_KERNEL_FFN2;
   Launch L(ctx, kind, s);
-  return ctx->cuda(launch_gemm_mx(ta, tb, p, kernel_epi, grid, s), "MXFP8 gemm launch");
+  return ctx->cuda(launch_gemm_mx(ta, tb, p, kernel_epi, grid, wide, s), "MXFP8 gemm launch");
 }
 
 h3dit_status run_attention(h3dit_ctx *ctx, const void *q, const void *k, const void *v, int ld,
@@ -491,26 +510,29 @@ h3dit_status run_unpack(h3dit_ctx *ctx, int n_txt, int n_img, void *x_txt, void 
 h3dit_status block_body_mx(h3dit_ctx *ctx, int l, const float *mod, int n, cudaStream_t s) {
   const int D = ctx->cfg.hidden, I = ctx->inner(), F = ctx->cfg.ffn;
   const MxWeights &o = ctx->L.wq_off;
+  auto tiled = [&](size_t off) -> const void * { return off == kNoTiled ? nullptr : ctx->wq(l, off); };
   uint8_t *xq = ctx->ws + ctx->L.xq, *xq_sf = ctx->ws + ctx->L.xq_sf;
   uint8_t *oq = ctx->ws + ctx->L.oq, *oq_sf = ctx->ws + ctx->L.oq_sf;
   uint8_t *uq = ctx->ws + ctx->L.uq, *uq_sf = ctx->ws + ctx->L.uq_sf;
   h3dit_status st = run_rmsnorm(ctx, ctx->resid(), mod, mod + D, xq, n, s, xq_sf);
   if (st) return st;
   if ((st = run_linear_mx(ctx, H3DIT_EPI_QKV_ROPE, xq, xq_sf, ctx->wq(l, o.qkv), ctx->wq(l, o.qkv_sf),
-                          n, 3 * I, D, ctx->qkv(), 3 * I, nullptr, nullptr, ctx->rope(), s)))
+                          n, 3 * I, D, ctx->qkv(), 3 * I, nullptr, nullptr, ctx->rope(), s,
+                          tiled(o.qkv_sft))))
     return st;
   const uint16_t *qkv = static_cast<const uint16_t *>(ctx->qkv());
   if ((st = run_attention(ctx, qkv, qkv + I, qkv + 2 * I, 3 * I, oq, I, n, s, oq_sf))) return st;
   if ((st = run_linear_mx(ctx, H3DIT_EPI_GATED_RESIDUAL, oq, oq_sf, ctx->wq(l, o.o), ctx->wq(l, o.o_sf),
-                          n, D, I, ctx->resid(), D, nullptr, mod + 2 * D, nullptr, s)))
+                          n, D, I, ctx->resid(), D, nullptr, mod + 2 * D, nullptr, s,
+                          tiled(o.o_sft))))
     return st;
   if ((st = run_rmsnorm(ctx, ctx->resid(), mod + 3 * D, mod + 4 * D, xq, n, s, xq_sf))) return st;
   if ((st = run_linear_mx(ctx, H3DIT_EPI_GELU, xq, xq_sf, ctx->wq(l, o.ff1), ctx->wq(l, o.ff1_sf), n,
-                          F, D, uq, F, uq_sf, nullptr, nullptr, s)))
+                          F, D, uq, F, uq_sf, nullptr, nullptr, s, tiled(o.ff1_sft))))
     return st;
   return run_linear_mx(ctx, H3DIT_EPI_GATED_RESIDUAL, uq, uq_sf, ctx->wq(l, o.ff2),
                        ctx->wq(l, o.ff2_sf), n, D, F, ctx->resid(), D, nullptr, mod + 5 * D,
-                       nullptr, s);
+                       nullptr, s, tiled(o.ff2_sft));
 }
 
 // Steps a3..a9 on the packed fp32 residual of n tokens (workspace).
@@ -632,6 +654,17 @@ h3dit_status h3dit_create(const h3dit_config *cfg, const h3dit_time_weights *tim
         e = launch_mx_quantize(b.w_ff1, D, F, D, ctx->wq(l, o.ff1), ctx->wq(l, o.ff1_sf), s);
       if (e == cudaSuccess)
         e = launch_mx_quantize(b.w_ff2, F, D, F, ctx->wq(l, o.ff2), ctx->wq(l, o.ff2_sf), s);
+      // and their scales repacked for the 224-column tiles
+      const struct {
+        size_t sf, sft;
+        int n, k;
+      } rep[4] = {{o.qkv_sf, o.qkv_sft, 3 * I, D},
+                  {o.o_sf, o.o_sft, D, I},
+                  {o.ff1_sf, o.ff1_sft, F, D},
+                  {o.ff2_sf, o.ff2_sft, D, F}};
+      for (int r = 0; r < 4 && e == cudaSuccess; ++r)
+        if (rep[r].sft != kNoTiled)
+          e = launch_mx_tile_sf(ctx->wq(l, rep[r].sf), rep[r].n, rep[r].k, ctx->wq(l, rep[r].sft), s);
     }
   }
   // the host vectors die with this call: the copies must have been consumed

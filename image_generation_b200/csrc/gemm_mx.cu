@@ -5,18 +5,24 @@
 // bf16 GEMM (RoPE on Q/K with a bf16 store, gated residual on the fp32
 // stream, and GELU written back as MXFP8 for the next linear).
 //
-// Structure (one CTA per SM, persistent over 128 x 128 output tiles):
-//   warp 0      TMA producer: A [128 x 128 B] and W [128 x 128 B] per k-block
-//               (128-byte swizzle) plus the two 512-byte scale blocks of that
-//               k-block (bulk copies), into a 6-stage shared-memory ring;
+// Structure (one CTA per SM, persistent over 128 x BN output tiles):
+//   warp 0      TMA producer: A [128 x 128 B] and W [BN x 128 B] per k-block
+//               (128-byte swizzle) plus that k-block's scale blocks (bulk
+//               copies), into a ring of shared-memory stages;
 //   warp 1      MMA issuer: per k-block, tcgen05.cp moves the A and W scale
 //               blocks into tensor memory (32x128b, copied to all four lane
 //               quarters), then 4 x tcgen05.mma.kind::mxf8f6f4.block_scale
-//               (M128 N128 K32) select scale byte kk of each 32-bit column;
+//               (M128 N=BN K32) select scale byte kk of each 32-bit column;
 //   warps 2..5  epilogue, as in the bf16 GEMM.
-// Tiles of 128 columns keep each W tile on one 128-row scale block and leave
-// tensor memory for two accumulators (2 x 128 columns) and the scale blocks of
-// every stage (6 x 8 columns).
+// Two tile widths:
+//   BN 128  W scales in the standard layout (one 512-byte block per 128 rows
+//           and k-block); two accumulators (2 x 128 columns) and the scales
+//           of six stages (6 x 8 columns) in tensor memory;
+//   BN 224  W scales repacked per tile (two 512-byte blocks covering rows
+//           224 t .. 224 t + 255 per k-block, made once when the weights are
+//           quantized); two accumulators (2 x 224 columns) and the scales of
+//           four stages (4 x 12 columns). An M128 N224 K32 MMA does 1.75x the
+//           work of an N128 one for about 1.3x its issue cost.
 #include "gemm_epilogue.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -26,22 +32,36 @@ namespace {
 
 using namespace gemm_detail;
 
-constexpr int BM = kGemmBM, BN = kGemmMxBN, BK = kGemmMxBK;
-constexpr int STAGES = 6;
-constexpr int A_BYTES = BM * BK;
-constexpr int B_BYTES = BN * BK;
-constexpr int SF_BYTES = 512;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + 2 * SF_BYTES;  // 33 KiB, keeps 1 KiB alignment
+constexpr int BM = kGemmBM, BK = kGemmMxBK;
 constexpr int THREADS = 192;
-constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + NUM_BARS * 8 + 16;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SF_COL0 = 2 * BN;  // scale blocks after the two accumulators
+constexpr int SF_BYTES = 512;
 
-template <int EPI>
+template <int BN>
+struct MxTile {
+  static constexpr bool WIDE = BN != kGemmMxBN;
+  static constexpr int STAGES = WIDE ? 4 : 6;
+  static constexpr int A_BYTES = BM * BK;
+  static constexpr int B_BYTES = BN * BK;
+  static constexpr int SFB_BYTES = WIDE ? 2 * SF_BYTES : SF_BYTES;
+  // stages keep 1 KiB alignment (128-byte swizzle atoms)
+  static constexpr int LOAD_BYTES = A_BYTES + B_BYTES + SF_BYTES + SFB_BYTES;  // per k-block
+  static constexpr int STAGE_BYTES = (LOAD_BYTES + 1023) / 1024 * 1024;
+  static constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + NUM_BARS * 8 + 16;
+  static constexpr uint32_t SF_COL0 = 2 * BN;        // scales after the two accumulators
+  static constexpr uint32_t SF_COLS = WIDE ? 12 : 8;  // per stage: A (4) then W (4 or 8)
+};
+static_assert(MxTile<kGemmMxWideBN>::SF_COL0 + 4 * 12 <= TMEM_COLS, "TMEM budget");
+static_assert(MxTile<kGemmMxWideBN>::SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+template <int EPI, int BN>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_mxf8_tcgen05(const __grid_constant__ CUtensorMap tma_a,
                       const __grid_constant__ CUtensorMap tma_b, const GemmParams p) {
+  using T = MxTile<BN>;
+  constexpr int STAGES = T::STAGES, A_BYTES = T::A_BYTES, B_BYTES = T::B_BYTES;
+  constexpr int STAGE_BYTES = T::STAGE_BYTES, NUM_BARS = T::NUM_BARS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -100,7 +120,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(FULL(stage), STAGE_BYTES);
+          mbar_arrive_expect_tx(FULL(stage), T::LOAD_BYTES);
           const uint32_t sa = sbase + stage * STAGE_BYTES;
           tma_load_2d(sa, &tma_a, kb * BK, tm * BM, FULL(stage));
           tma_load_2d(sa + A_BYTES, &tma_b, kb * BK, tn * BN, FULL(stage));
@@ -108,7 +128,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     p.a_sf + (static_cast<size_t>(tm) * kblocks + kb) * SF_BYTES, SF_BYTES,
                     FULL(stage));
           bulk_load(sa + A_BYTES + B_BYTES + SF_BYTES,
-                    p.b_sf + (static_cast<size_t>(tn) * kblocks + kb) * SF_BYTES, SF_BYTES,
+                    p.b_sf + (static_cast<size_t>(tn) * kblocks + kb) * T::SFB_BYTES, T::SFB_BYTES,
                     FULL(stage));
           ++issued;
           if (++stage == STAGES) {
@@ -147,10 +167,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc_fence_after();
           const uint32_t sa = sbase + stage * STAGE_BYTES;
           const uint32_t sb = sa + A_BYTES;
-          const uint32_t sfa_t = tmem + SF_COL0 + 8 * stage;
+          const uint32_t sfa_t = tmem + T::SF_COL0 + T::SF_COLS * stage;
           const uint32_t sfb_t = sfa_t + 4;
           tmem_cp_sf(sfa_t, desc_sf_copy(sb + B_BYTES));
           tmem_cp_sf(sfb_t, desc_sf_copy(sb + B_BYTES + SF_BYTES));
+          if (T::WIDE) tmem_cp_sf(sfb_t + 4, desc_sf_copy(sb + B_BYTES + 2 * SF_BYTES));
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
             const uint64_t da = desc_sw128(sa + kk * 32, 16, 1024);
@@ -200,18 +221,47 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int EPI>
+template <int EPI, int BN>
 cudaError_t launch_one(const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p, int grid,
                        cudaStream_t s) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_mxf8_tcgen05<EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(gemm_mxf8_tcgen05<EPI, BN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         MxTile<BN>::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  gemm_mxf8_tcgen05<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(a, b, p);
+  gemm_mxf8_tcgen05<EPI, BN><<<grid, THREADS, MxTile<BN>::SMEM_BYTES, s>>>(a, b, p);
   return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_bn(const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p, int grid,
+                      bool wide, cudaStream_t s) {
+  return wide ? launch_one<EPI, kGemmMxWideBN>(a, b, p, grid, s)
+              : launch_one<EPI, kGemmMxBN>(a, b, p, grid, s);
+}
+
+// Repack W scales (standard layout) for 224-row tiles: byte i of the output
+// belongs to tile i / (kb * 1024), k-block (i / 1024) % kb, half (i / 512) % 2
+// and, inside that 512-byte block, row r and scale j of the standard in-block
+// order; rows past n read as zero.
+__global__ void mx_tile_sf_kernel(const uint8_t *__restrict__ sf, int n, int k,
+                                  uint8_t *__restrict__ tiled, long long total) {
+  const int kblocks = k / 128;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long blk = i / 512;
+    const int within = static_cast<int>(i % 512);
+    const int half = static_cast<int>(blk % 2);
+    const int kb = static_cast<int>((blk / 2) % kblocks);
+    const long long tile = blk / 2 / kblocks;
+    const int r = within / 16 + 32 * ((within % 16) / 4);
+    const int j = within % 4;
+    const long long row = tile * kGemmMxWideBN + 128 * half + r;
+    tiled[i] = row < n ? sf[mx_sf_offset(static_cast<int>(row), 4 * kb + j, kblocks)] : 0;
+  }
 }
 
 // One thread per block of 32 consecutive elements of a row: bf16 in,
@@ -248,19 +298,28 @@ __global__ void mx_quantize_kernel(const uint16_t *__restrict__ src, long long l
 }  // namespace
 
 cudaError_t launch_gemm_mx(const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p,
-                           int epilogue, int grid, cudaStream_t s) {
+                           int epilogue, int grid, bool wide, cudaStream_t s) {
   switch (epilogue) {
     case kEpiQkvRope:
-      return launch_one<kEpiQkvRope>(a, b, p, grid, s);
+      return launch_bn<kEpiQkvRope>(a, b, p, grid, wide, s);
     case kEpiGatedResidual:
-      return launch_one<kEpiGatedResidual>(a, b, p, grid, s);
+      return launch_bn<kEpiGatedResidual>(a, b, p, grid, wide, s);
     case kEpiGeluMx:
-      return launch_one<kEpiGeluMx>(a, b, p, grid, s);
+      return launch_bn<kEpiGeluMx>(a, b, p, grid, wide, s);
     case kEpiStore:
-      return launch_one<kEpiStore>(a, b, p, grid, s);
+      return launch_bn<kEpiStore>(a, b, p, grid, wide, s);
     default:
       return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_mx_tile_sf(const uint8_t *sf, int n, int k, uint8_t *tiled, cudaStream_t s) {
+  const long long total = static_cast<long long>(mx_sf_tiled_bytes(n, k));
+  if (total <= 0) return cudaSuccess;
+  const long long want = (total + 255) / 256;
+  const int grid = static_cast<int>(want < 148LL * 16 ? want : 148LL * 16);
+  mx_tile_sf_kernel<<<grid, 256, 0, s>>>(sf, n, k, tiled, total);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_mx_quantize(const void *src, long long ld, int rows, int k, uint8_t *dst,

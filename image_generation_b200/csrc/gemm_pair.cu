@@ -16,7 +16,7 @@
 //               takes one arrival (with its byte count) from each producer;
 //   warp 1      TMEM allocation for the pair; in the first CTA only, the MMA
 //               issuer: 4 pair MMAs per k-block into one of two 256-column
-//               accumulators, commits multicast to both CTAs' EMPTY / TFULL;
+//               accumulators; each commit arrives on both CTAs' EMPTY / TFULL;
 //   warps 2..5  epilogue of this CTA's 128 rows, unchanged from the one-CTA
 //               kernel; every thread then arrives on the first CTA's TEMPTY.
 //
@@ -44,7 +44,7 @@ constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + NUM_BARS * 8 + 16;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC = idesc_bf16_f32(2 * BM, BN, false, false);
-constexpr uint16_t BOTH = 0x3;
+constexpr uint16_t kBothCtas = 0x3, kFirstCta = 0x1;
 
 template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -168,20 +168,20 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint64_t db = desc_sw128(sb + kk * 32, 16, 1024);
             umma_bf16_pair(d, da, db, IDESC, (kb | kk) != 0 ? 1u : 0u);
           }
-          umma_commit_pair(EMPTY(stage), BOTH);
+          umma_commit_pair(EMPTY(stage), kBothCtas);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        umma_commit_pair(TFULL(acc), BOTH);
+        umma_commit_pair(TFULL(acc), kBothCtas);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1;
       }
       // Every pair MMA (and the arrivals its commits make) completes before
       // either CTA may release TMEM or exit.
-      umma_commit_pair(DRAIN, 0x1);
+      umma_commit_pair(DRAIN, kFirstCta);
       mbar_wait(DRAIN, 0, p.status, false);
     }
   } else {

@@ -90,8 +90,16 @@ cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const C
 // W [n, k] as E4M3 with scales in the mx_sf layout.
 constexpr int kGemmMxBN = 128;
 constexpr int kGemmMxBK = 128;
+// Wide tiles (128 x 224) take W scales repacked per tile: for tile t and
+// k-block kb, the two 512-byte blocks of rows 224 t .. 224 t + 127 and
+// 224 t + 128 .. 224 t + 255 (standard in-block order) at (t * (k/128) + kb) * 1024.
+constexpr int kGemmMxWideBN = 224;
+inline size_t mx_sf_tiled_bytes(long long n, long long k) {
+  return static_cast<size_t>(n / kGemmMxWideBN) * static_cast<size_t>(k / 128) * 1024;
+}
 cudaError_t launch_gemm_mx(const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p,
-                           int epilogue, int grid, cudaStream_t s);
+                           int epilogue, int grid, bool wide, cudaStream_t s);
+cudaError_t launch_mx_tile_sf(const uint8_t *sf, int n, int k, uint8_t *tiled, cudaStream_t s);
 // bf16 [rows, k] (row stride ld elements) -> E4M3 [rows, k] + scales.
 cudaError_t launch_mx_quantize(const void *src, long long ld, int rows, int k, uint8_t *dst,
                                uint8_t *sf, cudaStream_t s);

@@ -142,7 +142,7 @@ def _quantized(ctx, a):
     return q.view(rows, k), sf
 
 
-@pytest.mark.parametrize("m", [1, 200])
+@pytest.mark.parametrize("m", [1, 200, 300])
 @pytest.mark.parametrize("n,k", [(768, 768), (2048, 768), (768, 2048)])
 def test_linear_mx_epilogues(small, m, n, k):
     from image_generation_b200 import h3dit as H
@@ -168,13 +168,33 @@ def test_linear_mx_epilogues(small, m, n, k):
     assert_mx_bound(codes, X, O.gelu(ref), "linear mx gelu (MXFP8 out)")
 
 
+@pytest.mark.parametrize("k", [128, 256])
+def test_linear_mx_several_tiles_per_cta(small, k):
+    """More output tiles than CTAs (pairs): several tiles per persistent CTA
+    through both accumulators and the scale columns of every stage; a ragged
+    last row block; fewer k-blocks than stages."""
+    from image_generation_b200 import h3dit as H
+
+    m, n = 4500, 2048
+    a = synth.tokens(m, k, 7 + k, "a")
+    w = synth.normal_bf16((n, k), 0.02, 7 + k, "w")
+    aq, asf = _quantized(small, a)
+    wq, wsf = _quantized(small, w)
+    out = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+    small.linear_mx(H.H3DIT_EPI_STORE, aq, asf, wq, wsf, out)
+    torch.cuda.synchronize()
+    assert small.sync_status() == 0
+    assert_close(to_np(out), O.linear_mx(a, w), "linear mx, many tiles", cos_min=0.99999)
+
+
+@pytest.mark.parametrize("grids", [[(0, 9, 11)], [(0, 16, 17)]], ids=["104tok", "277tok"])
 @pytest.mark.parametrize("dims", [synth.SMALL, synth.Dims(768, 6, 128, 2048)], ids=["d96", "d128"])
-def test_linear_mx_qkv_rope(dims):
+def test_linear_mx_qkv_rope(dims, grids):
     from image_generation_b200 import h3dit as H
 
     ctx, _, bws = _ctx(dims)
     ocfg = O.config_for(dims.hidden, dims.heads, dims.head_dim, dims.ffn)
-    grids, n_txt = [(0, 9, 11)], 5
+    n_txt = 5
     pos = O.token_positions(n_txt, grids)
     m = pos.shape[0]
     xm = synth.tokens(m, dims.hidden, 4, "xm")
@@ -235,6 +255,18 @@ def test_block_mx_small(dims):
     y, x, ref = _block_mx_case(dims, 32, [(0, 16, 16)], 8)
     assert_close(y, ref, "MXFP8 block", cos_min=MX_COS, rel_max=np.inf)
     assert_delta_close(y - x, ref - x, "MXFP8 block (branch delta)", cos_min=MX_COS, row_cos_min=0.99)
+
+
+def test_block_mx_wide_tiles():
+    """Hidden 2688 (28 heads x 96), FFN 3584: every linear's N is a multiple
+    of 224, so the block runs all four on the wide (128 x 224) tiles with the
+    W scales repacked per tile; 21 text + 18 x 17 image tokens span several
+    row blocks with a ragged last one."""
+    dims = synth.Dims(2688, 28, 96, 3584)
+    y, x, ref = _block_mx_case(dims, 21, [(0, 18, 17)], 5)
+    assert_close(y, ref, "MXFP8 block, wide tiles", cos_min=MX_COS, rel_max=np.inf)
+    assert_delta_close(y - x, ref - x, "MXFP8 block, wide tiles (branch delta)", cos_min=MX_COS,
+                       row_cos_min=0.99)
 
 
 def test_block_mx_full_width_4k_sampled_rows():
