@@ -97,19 +97,58 @@ H3_DEV constexpr bool use_poly(int pair) {
   return EMU == 1 ? (pair % 4) == 3 : EMU == 2 ? (pair % 2) == 1 : false;
 }
 
-// TMEM loads / stores of a row's scores (BKV columns) and packed P (BKV/2).
-template <int N>
-H3_DEV void tmem_ld_n(uint32_t taddr, uint32_t (&r)[N]);
-template <>
-H3_DEV void tmem_ld_n<64>(uint32_t taddr, uint32_t (&r)[64]) { tmem_ld64(taddr, r); }
-template <>
-H3_DEV void tmem_ld_n<128>(uint32_t taddr, uint32_t (&r)[128]) { tmem_ld128(taddr, r); }
-template <int N>
-H3_DEV void tmem_st_n(uint32_t taddr, const uint32_t (&r)[N]);
-template <>
-H3_DEV void tmem_st_n<32>(uint32_t taddr, const uint32_t (&r)[32]) { tmem_st32(taddr, r); }
-template <>
-H3_DEV void tmem_st_n<64>(uint32_t taddr, const uint32_t (&r)[64]) { tmem_st64(taddr, r); }
+// One row's scores for 64 keys from TMEM; keys at or past `valid` are -inf
+// (only the last KV tile has any).
+H3_DEV void load_scores64(uint32_t taddr, float (&s)[64], int valid) {
+  uint32_t r[64];
+  tmem_ld64(taddr, r);
+#pragma unroll
+  for (int i = 0; i < 64; ++i) s[i] = __uint_as_float(r[i]);
+  if (valid < 64) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i)
+      if (i >= valid) s[i] = -INFINITY;
+  }
+}
+
+// Max of 64 scores: eight independent chains (a two-input max, then three
+// three-input maxes each), then a three-level combine.
+H3_DEV float row_max64(const float (&s)[64]) {
+  float a[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) a[c] = fmaxf(s[c], s[8 + c]);
+#pragma unroll
+  for (int i = 16; i < 64; i += 16) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) a[c] = fmax3(a[c], s[i + c], s[i + 8 + c]);
+  }
+  return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+}
+
+// p_i = 2^(s_i * scale_log2 - m) for 64 scores, two at a time: added into the
+// four partial row sums and packed as bf16 pairs (the A operand of PV).
+template <int DH>
+H3_DEV void exp_pack64(const float (&s)[64], float sl2, float m, uint64_t (&part)[4],
+                       uint32_t (&pk)[32]) {
+  const uint64_t sl2x2 = f2_pack(sl2, sl2);
+  const uint64_t negm2 = f2_pack(-m, -m);
+#pragma unroll
+  for (int i = 0; i < 64; i += 2) {
+    const uint64_t y2 = f2_fma(f2_pack(s[i], s[i + 1]), sl2x2, negm2);
+    uint64_t e2;
+    if (use_poly<kExpEmu<DH>>(i / 2)) {
+      e2 = exp2_poly2(y2);
+    } else {
+      float y0, y1;
+      f2_unpack(y2, y0, y1);
+      e2 = f2_pack(ex2_approx(y0), ex2_approx(y1));
+    }
+    part[(i / 2) & 3] = f2_add(part[(i / 2) & 3], e2);
+    float e0, e1;
+    f2_unpack(e2, e0, e1);
+    pk[i / 2] = pack_bf16x2(e0, e1);
+  }
+}
 
 // O_t (+)= P_t V with P_t in TMEM (kind::f16, A from tensor memory).
 H3_DEV void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
@@ -246,8 +285,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t v_src = sKV + (j % NS) * STAGE_BYTES + KV_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk) {
-          // A: P_t(j) in TMEM, 16 keys = 8 packed columns per step
-          umma_bf16_ts(o_tmem, s_base + static_cast<uint32_t>(BKV * (j % SBUF)) + 8 * kk,
+          // A: P_t(j) in TMEM, 16 keys = 8 packed columns per step (with
+          // 128 keys, keys 64..127 sit in columns 64..95)
+          const uint32_t p_col = 8 * kk + (kk >= 4 ? 32 : 0);
+          umma_bf16_ts(o_tmem, s_base + static_cast<uint32_t>(BKV * (j % SBUF)) + p_col,
                        desc_sw128(v_src + kk * 16 * 128, KBOX, 1024), IDESC_O,
                        (j > 0 || kk > 0) ? 1u : 0u);
         }
@@ -281,58 +322,52 @@ __global__ void __launch_bounds__(THREADS, 1)
         break;
       }
       tc_fence_after();
-      float s[BKV];
-      {
-        uint32_t r[BKV];
-        tmem_ld_n<BKV>(tS, r);
-#pragma unroll
-        for (int i = 0; i < BKV; ++i) s[i] = __uint_as_float(r[i]);
-      }
-      const int valid = p.n - j * BKV;
-      if (valid < BKV) {
-#pragma unroll
-        for (int i = 0; i < BKV; ++i)
-          if (i >= valid) s[i] = -INFINITY;
-      }
-      // row max: eight independent chains of three-input max, then combine
-      float a8[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) a8[c] = s[c];
-#pragma unroll
-      for (int i = 8; i < BKV; i += 16) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) a8[c] = fmax3(a8[c], s[i + c], s[i + 8 + c]);
-      }
-      float mx = fmax3(fmax3(a8[0], a8[1], a8[2]), fmax3(a8[3], a8[4], a8[5]), fmaxf(a8[6], a8[7]));
-      mx *= sl2;
+      const int valid = p.n - j * BKV;  // keys of this tile that exist
       float alpha = 1.f;
       bool rescale = false;
-      if (j == 0) {
-        m = mx;
-      } else if (mx > m + RESCALE_THRESHOLD) {
-        alpha = ex2_approx(m - mx);
-        m = mx;
-        rescale = true;
-      }
-      const uint64_t sl2x2 = f2_pack(sl2, sl2);
-      const uint64_t negm2 = f2_pack(-m, -m);
-      uint64_t part[4] = {0, 0, 0, 0};
-      uint32_t pk[BKV / 2];
-#pragma unroll
-      for (int i = 0; i < BKV; i += 2) {
-        const uint64_t y2 = f2_fma(f2_pack(s[i], s[i + 1]), sl2x2, negm2);
-        uint64_t e2;
-        if (use_poly<kExpEmu<DH>>(i / 2)) {
-          e2 = exp2_poly2(y2);
-        } else {
-          float y0, y1;
-          f2_unpack(y2, y0, y1);
-          e2 = f2_pack(ex2_approx(y0), ex2_approx(y1));
+      auto update_max = [&](float mx) {  // mx: row max of the raw scores
+        mx *= sl2;
+        if (j == 0) {
+          m = mx;
+        } else if (mx > m + RESCALE_THRESHOLD) {
+          alpha = ex2_approx(m - mx);
+          m = mx;
+          rescale = true;
         }
-        part[(i / 2) & 3] = f2_add(part[(i / 2) & 3], e2);
-        float e0, e1;
-        f2_unpack(e2, e0, e1);
-        pk[i / 2] = pack_bf16x2(e0, e1);
+      };
+      uint64_t part[4] = {0, 0, 0, 0};
+      if constexpr (BKV == 64) {
+        float sc[64];
+        load_scores64(tS, sc, valid);
+        update_max(row_max64(sc));
+        uint32_t pk[32];
+        exp_pack64<DH>(sc, sl2, m, part, pk);
+        tmem_st32(tS, pk);
+      } else {
+        // 128 keys in two halves of 64 columns, read twice from TMEM (a
+        // second read is cheaper than holding 128 scores in registers): the
+        // max over both halves, then each half's P over its own scores, keys
+        // 64..127 to columns 64..95 first, then keys 0..63 to columns 0..31.
+        float mx_lo;
+        {
+          float lo[64];
+          load_scores64(tS, lo, valid);
+          mx_lo = row_max64(lo);
+        }
+        asm volatile("" : "+f"(mx_lo));  // the first half is reduced before the second loads
+        {
+          float hi[64];
+          load_scores64(tS + 64, hi, valid - 64);
+          update_max(fmaxf(mx_lo, row_max64(hi)));
+        }
+#pragma unroll 1
+        for (int h = 64; h >= 0; h -= 64) {
+          float sc[64];
+          load_scores64(tS + h, sc, valid - h);
+          uint32_t pk[32];
+          exp_pack64<DH>(sc, sl2, m, part, pk);
+          tmem_st32(tS + h, pk);
+        }
       }
       float sum;
       {
@@ -359,7 +394,6 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_st32(tO + 32 * c, r);
         }
       }
-      tmem_st_n<BKV / 2>(tS, pk);
       tc_fence_before();
       mbar_arrive(P_FULL(t, j % SBUF));
     }
