@@ -341,13 +341,16 @@ def run_only(args):
     dh = args.head_dim
     I = H * dh
     torch.manual_seed(0)
-    cfg = Hb.make_config(D, H, dh, F, 1, N_TOK)
+    mx = bool(args.mx) and args.only in ("qkv", "out_proj", "ffn1", "ffn2")
+    cfg = Hb.make_config(D, H, dh, F, 1, N_TOK,
+                         precision=Hb.H3DIT_PRECISION_MXFP8 if mx else Hb.H3DIT_PRECISION_BF16)
     g = lambda *s: (torch.randn(*s, device="cuda") * 0.02).bfloat16()
     tw = {"w_t1": torch.randn(D, 256, device="cuda") * 0.02, "b_t1": torch.zeros(D, device="cuda"),
           "w_t2": torch.randn(D, D, device="cuda") * 0.02, "b_t2": torch.zeros(D, device="cuda")}
     need = {"qkv": "w_qkv", "out_proj": "w_o", "ffn1": "w_ff1", "ffn2": "w_ff2"}.get(args.only)
     shapes = {"w_qkv": (3 * I, D), "w_o": (D, I), "w_ff1": (F, D), "w_ff2": (D, F), "w_ada": (6 * D, D)}
-    blk = {k: (g(*shp) if k in (need, "w_ada") else torch.zeros(8, device="cuda").bfloat16())
+    # an MXFP8 context quantizes all four linears at create: they must be full size
+    blk = {k: (g(*shp) if k in (need, "w_ada") or mx else torch.zeros(8, device="cuda").bfloat16())
            for k, shp in shapes.items()}
     blk["b_ada"] = torch.zeros(6 * D, device="cuda")
     ctx = Hb.Context(cfg, tw, [blk])
@@ -356,29 +359,29 @@ def run_only(args):
         qkv = torch.randn(n, 3 * I, device="cuda").bfloat16()
         o = torch.empty(n, I, device="cuda", dtype=torch.bfloat16)
         fn = lambda: ctx.attention(qkv[:, :I], qkv[:, I:2 * I], qkv[:, 2 * I:], 3 * I, o, I, n)
-    elif args.mx and args.only in ("qkv", "ffn1", "out_proj", "ffn2"):
+    elif mx:
+        # the block's own MXFP8 linear (weights quantized at create), through
+        # the kernel the MXFP8 step runs for it
         w = blk[need]
         a = torch.randn(n, w.shape[1], device="cuda").bfloat16()
-        aq = torch.empty(n * w.shape[1], dtype=torch.uint8, device="cuda")
+        aq = torch.empty(n, w.shape[1], dtype=torch.uint8, device="cuda")
         asf = torch.empty(Hb.mx_scale_bytes(n, w.shape[1]), dtype=torch.uint8, device="cuda")
-        wq = torch.empty(w.numel(), dtype=torch.uint8, device="cuda")
-        wsf = torch.empty(Hb.mx_scale_bytes(w.shape[0], w.shape[1]), dtype=torch.uint8, device="cuda")
         ctx.mx_quantize(a, aq, asf)
-        ctx.mx_quantize(w, wq, wsf)
-        aq, wq = aq.view(n, -1), wq.view(w.shape[0], -1)
+        which = {"qkv": Hb.H3DIT_LINEAR_QKV, "out_proj": Hb.H3DIT_LINEAR_OUT,
+                 "ffn1": Hb.H3DIT_LINEAR_FFN1, "ffn2": Hb.H3DIT_LINEAR_FFN2}[args.only]
         if args.only == "qkv":
             table = torch.empty(n, dh // 2, 2, device="cuda")
             ctx.rope_table([(0, GRID, GRID)], N_TXT, table)
             out = torch.empty(n, w.shape[0], device="cuda", dtype=torch.bfloat16)
-            fn = lambda: ctx.linear_mx(Hb.H3DIT_EPI_QKV_ROPE, aq, asf, wq, wsf, out, rope_table=table)
+            fn = lambda: ctx.block_linear_mx(0, which, aq, asf, out, rope_table=table)
         elif args.only == "ffn1":
-            out = torch.empty(n * w.shape[0], device="cuda", dtype=torch.uint8)
+            out = torch.empty(n, w.shape[0], device="cuda", dtype=torch.uint8)
             osf = torch.empty(Hb.mx_scale_bytes(n, w.shape[0]), dtype=torch.uint8, device="cuda")
-            fn = lambda: ctx.linear_mx(Hb.H3DIT_EPI_GELU, aq, asf, wq, wsf, out, out_sf=osf)
+            fn = lambda: ctx.block_linear_mx(0, which, aq, asf, out, out_sf=osf)
         else:
             x = torch.randn(n, D, device="cuda")
             gate = torch.full((D,), 0.1, device="cuda")
-            fn = lambda: ctx.linear_mx(Hb.H3DIT_EPI_GATED_RESIDUAL, aq, asf, wq, wsf, x, gate=gate)
+            fn = lambda: ctx.block_linear_mx(0, which, aq, asf, x, gate=gate)
     elif args.only in ("qkv", "ffn1"):
         xm = torch.randn(n, D, device="cuda").bfloat16()
         table = torch.empty(n, dh // 2, 2, device="cuda")

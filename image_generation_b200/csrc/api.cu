@@ -833,6 +833,41 @@ h3dit_status h3dit_linear_mx(h3dit_ctx *ctx, int32_t epilogue, const void *a, co
                        static_cast<cudaStream_t>(cuda_stream));
 }
 
+h3dit_status h3dit_block_linear_mx(h3dit_ctx *ctx, int32_t block, int32_t which, const void *a,
+                                   const void *a_sf, int32_t m, void *out, void *out_sf,
+                                   const float *gate, const float *rope_table, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (!ctx->mx()) return ctx->fail(H3DIT_ERR_UNSUPPORTED, "the context is not MXFP8");
+  if (block < 0 || block >= ctx->cfg.n_blocks)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "block %d outside [0, %d)", block, ctx->cfg.n_blocks);
+  const int D = ctx->cfg.hidden, I = ctx->inner(), F = ctx->cfg.ffn;
+  const MxWeights &o = ctx->L.wq_off;
+  auto tiled = [&](size_t off) -> const void * {
+    return off == kNoTiled ? nullptr : ctx->wq(block, off);
+  };
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  switch (which) {
+    case H3DIT_LINEAR_QKV:
+      return run_linear_mx(ctx, H3DIT_EPI_QKV_ROPE, a, a_sf, ctx->wq(block, o.qkv),
+                           ctx->wq(block, o.qkv_sf), m, 3 * I, D, out, 3 * I, nullptr, nullptr,
+                           rope_table, s, tiled(o.qkv_sft));
+    case H3DIT_LINEAR_OUT:
+      return run_linear_mx(ctx, H3DIT_EPI_GATED_RESIDUAL, a, a_sf, ctx->wq(block, o.o),
+                           ctx->wq(block, o.o_sf), m, D, I, out, D, nullptr, gate, nullptr, s,
+                           tiled(o.o_sft));
+    case H3DIT_LINEAR_FFN1:
+      return run_linear_mx(ctx, H3DIT_EPI_GELU, a, a_sf, ctx->wq(block, o.ff1),
+                           ctx->wq(block, o.ff1_sf), m, F, D, out, F, out_sf, nullptr, nullptr, s,
+                           tiled(o.ff1_sft));
+    case H3DIT_LINEAR_FFN2:
+      return run_linear_mx(ctx, H3DIT_EPI_GATED_RESIDUAL, a, a_sf, ctx->wq(block, o.ff2),
+                           ctx->wq(block, o.ff2_sf), m, D, F, out, D, nullptr, gate, nullptr, s,
+                           tiled(o.ff2_sft));
+    default:
+      return ctx->fail(H3DIT_ERR_INVALID_ARG, "unknown linear %d", which);
+  }
+}
+
 h3dit_status h3dit_rmsnorm_modulate_mx(h3dit_ctx *ctx, const float *x, const float *shift,
                                        const float *scale, void *out, void *out_sf, int32_t n,
                                        void *cuda_stream) {

@@ -28,6 +28,11 @@ H3DIT_EPI_QKV_ROPE = 1
 H3DIT_EPI_GELU = 2
 H3DIT_EPI_GATED_RESIDUAL = 3
 
+H3DIT_LINEAR_QKV = 0
+H3DIT_LINEAR_OUT = 1
+H3DIT_LINEAR_FFN1 = 2
+H3DIT_LINEAR_FFN2 = 3
+
 H3DIT_PRECISION_BF16 = 0
 H3DIT_PRECISION_MXFP8 = 1
 H3DIT_STATIC_TIME_MAX_HIDDEN = 8192
@@ -92,6 +97,7 @@ def _load() -> C.CDLL:
         "h3dit_mx_scale_bytes": (sz, [i32, i32]),
         "h3dit_mx_quantize": (i32, [p, p, i32, i32, p, p, p]),
         "h3dit_linear_mx": (i32, [p, i32, p, p, p, p, i32, i32, i32, p, p, p, p, p]),
+        "h3dit_block_linear_mx": (i32, [p, i32, i32, p, p, i32, p, p, p, p, p]),
         "h3dit_rmsnorm_modulate_mx": (i32, [p, p, p, p, p, p, i32, p]),
         "h3dit_attention_mx": (i32, [p, p, p, p, i32, p, p, i32, p]),
         "h3dit_selftest_bounded_wait": (i32, [p, i32, p]),
@@ -252,6 +258,12 @@ class Context:
         self._check(lib.h3dit_linear_mx(self.handle, epilogue, _ptr(a), _ptr(a_sf), _ptr(w),
                                         _ptr(w_sf), m, n, k, _ptr(out), _ptr(out_sf), _ptr(gate),
                                         _ptr(rope_table), _stream(stream)))
+
+    def block_linear_mx(self, block: int, which: int, a, a_sf, out, out_sf=None, gate=None,
+                        rope_table=None, stream=None) -> None:
+        self._check(lib.h3dit_block_linear_mx(self.handle, block, which, _ptr(a), _ptr(a_sf),
+                                              a.shape[0], _ptr(out), _ptr(out_sf), _ptr(gate),
+                                              _ptr(rope_table), _stream(stream)))
 
     def rmsnorm_modulate_mx(self, x, shift, scale, out, out_sf, stream=None) -> None:
         self._check(lib.h3dit_rmsnorm_modulate_mx(self.handle, _ptr(x), _ptr(shift), _ptr(scale),

@@ -221,6 +221,24 @@ h3dit_status h3dit_linear_mx(h3dit_ctx *ctx, int32_t epilogue, const void *a, co
                              void *out, void *out_sf, const float *gate, const float *rope_table,
                              void *cuda_stream);
 
+/* The block's four linears, for h3dit_block_linear_mx. */
+#define H3DIT_LINEAR_QKV 0  /* QKV + RoPE:            out bf16 [m, 3*heads*head_dim] */
+#define H3DIT_LINEAR_OUT 1  /* out-proj, gated:       out fp32 [m, hidden] += gate * acc */
+#define H3DIT_LINEAR_FFN1 2 /* FFN1 + GELU to MXFP8:  out E4M3 [m, ffn] + out_sf */
+#define H3DIT_LINEAR_FFN2 3 /* FFN2, gated:           out fp32 [m, hidden] += gate * acc */
+
+/* One of block `block`'s MXFP8 linears on the context's own quantized
+ * weights (precision H3DIT_PRECISION_MXFP8 only), with that linear's
+ * epilogue and through exactly the kernel h3dit_block_forward runs for it:
+ * 128 x 224 tiles with the weight scales repacked per tile where N is a
+ * multiple of 224 and every tile starts on a rotary-section boundary, else
+ * 128 x 128 tiles. `a` E4M3 [m, k] + a_sf (h3dit_mx_scale_bytes(m, k)), k the
+ * linear's input width; rope_table for H3DIT_LINEAR_QKV, gate for OUT and
+ * FFN2, out_sf for FFN1. Returns H3DIT_ERR_UNSUPPORTED on a bf16 context. */
+h3dit_status h3dit_block_linear_mx(h3dit_ctx *ctx, int32_t block, int32_t which, const void *a,
+                                   const void *a_sf, int32_t m, void *out, void *out_sf,
+                                   const float *gate, const float *rope_table, void *cuda_stream);
+
 /* a3/a7 with an MXFP8 output: out E4M3 [n, D] + out_sf. */
 h3dit_status h3dit_rmsnorm_modulate_mx(h3dit_ctx *ctx, const float *x, const float *shift,
                                        const float *scale, void *out, void *out_sf, int32_t n,

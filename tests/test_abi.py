@@ -113,6 +113,8 @@ def test_null_context_is_rejected_everywhere():
         == H.H3DIT_ERR_INVALID_ARG
     assert H.lib.h3dit_attention(None, 0x10000, 0x10000, 0x10000, 768, 0x10000, 768, 4, None) \
         == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_block_linear_mx(None, 0, H.H3DIT_LINEAR_QKV, 0x10000, 0x10000, 4, 0x10000,
+                                       None, None, 0x10000, None) == H.H3DIT_ERR_INVALID_ARG
     H.lib.h3dit_destroy(None)  # NULL-safe
     assert H.lib.h3dit_last_error(None) == b"no context"
 

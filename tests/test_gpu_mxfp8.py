@@ -269,6 +269,55 @@ def test_block_mx_wide_tiles():
                        row_cos_min=0.99)
 
 
+@pytest.mark.parametrize("dims", [synth.Dims(2688, 28, 96, 3584), synth.SMALL, synth.Dims(768, 6, 128, 2048)],
+                         ids=["wide_d96", "narrow_d96", "narrow_d128"])
+def test_block_linear_mx_stages(dims):
+    """Each of a block's MXFP8 linears through the stage entry point, on the
+    context's own quantized weights: wide (128 x 224) tiles where every N is
+    a multiple of 224 (hidden 2688), the 128-wide kernel otherwise."""
+    from image_generation_b200 import h3dit as H
+
+    ctx, _, bws = _ctx(dims, max_tokens=300, precision=1)
+    ocfg = O.config_for(dims.hidden, dims.heads, dims.head_dim, dims.ffn)
+    I, D, F = ocfg.inner, dims.hidden, dims.ffn
+    bw = bws[0]
+    grids, n_txt = [(0, 11, 19)], 9
+    pos = O.token_positions(n_txt, grids)
+    m = pos.shape[0]
+    # QKV + RoPE
+    x = synth.tokens(m, D, 21, "x")
+    xq, xsf = _quantized(ctx, x)
+    table = torch.empty(m, dims.head_dim // 2, 2, dtype=torch.float32, device="cuda")
+    ctx.rope_table(grids, n_txt, table)
+    qkv = torch.empty(m, 3 * I, dtype=torch.bfloat16, device="cuda")
+    ctx.block_linear_mx(0, H.H3DIT_LINEAR_QKV, xq, xsf, qkv, rope_table=table)
+    y = O.linear_mx(x, bw["w_qkv"])
+    q = O.apply_rope(y[:, :I].reshape(m, -1, dims.head_dim), pos, ocfg.rope_sections, 1e4)
+    k = O.apply_rope(y[:, I:2 * I].reshape(m, -1, dims.head_dim), pos, ocfg.rope_sections, 1e4)
+    ref = np.concatenate([q.reshape(m, -1), k.reshape(m, -1), y[:, 2 * I:]], axis=1)
+    # out-projection and FFN2 with the gated residual, FFN1 to MXFP8
+    a = synth.tokens(m, I, 22, "a")
+    aq, asf = _quantized(ctx, a)
+    u = synth.tokens(m, F, 23, "u")
+    uq, usf = _quantized(ctx, u)
+    r0 = synth.normal_f32((m, D), 1.0, 24, "r")
+    gate = synth.normal_f32((D,), 0.3, 24, "g")
+    r_out, r_ff2 = to_dev(r0, "f32"), to_dev(r0, "f32")
+    ctx.block_linear_mx(0, H.H3DIT_LINEAR_OUT, aq, asf, r_out, gate=to_dev(gate, "f32"))
+    ctx.block_linear_mx(0, H.H3DIT_LINEAR_FFN2, uq, usf, r_ff2, gate=to_dev(gate, "f32"))
+    hq, hsf = _alloc_mx(m, F)
+    ctx.block_linear_mx(0, H.H3DIT_LINEAR_FFN1, xq, xsf, hq, out_sf=hsf)
+    torch.cuda.synchronize()
+    assert ctx.sync_status() == 0
+    assert_close(to_np(qkv), ref, "block QKV mx + rope", cos_min=0.99999)
+    assert_close(to_np(r_out) - r0, gate * O.linear_mx(a, bw["w_o"]), "block out-proj mx",
+                 cos_min=0.99999, rel_max=1e-3)
+    assert_close(to_np(r_ff2) - r0, gate * O.linear_mx(u, bw["w_ff2"]), "block FFN2 mx",
+                 cos_min=0.99999, rel_max=1e-3)
+    codes, X = _decode(hq, hsf, m, F)
+    assert_mx_bound(codes, X, O.gelu(O.linear_mx(x, bw["w_ff1"])), "block FFN1 mx gelu")
+
+
 def test_block_mx_full_width_4k_sampled_rows():
     w = synth.WORKLOADS["block_4k"]
     rows = np.unique(np.concatenate([np.arange(24), np.random.default_rng(3).choice(
