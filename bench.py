@@ -6,7 +6,11 @@
     python bench.py --impl reference          # the CPU oracle on a bounded sample
     python bench.py --only attention          # one kernel kind alone (for profilers)
 
-Rank 0 prints one JSON line. Multi-GPU runs are independent replicas (the
+Rank 0 prints one JSON line. Besides the contract's keys it carries the
+per-step median/min/max, the same step replayed from a CUDA graph, the 6-step
+total, the GEMM and attention TFLOP/s, ms per block at the other workload
+shapes (small block, 2048^2, 4096^2, the edit request with four references)
+and the MXFP8 variant of the step. Multi-GPU runs are independent replicas (the
 step does not shard): every rank runs its own step on its own weights, the
 timed region is bracketed by barriers and the slowest rank's time is used.
 Weights are random-init bf16 (44 GB for 50 blocks at head_dim 96), generated
@@ -39,7 +43,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="h3dit", choices=["h3dit", "reference"])
     ap.add_argument("--head-dim", type=int, default=96, choices=[96, 128])
@@ -48,6 +52,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-mxfp8", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the graph-replayed step timing")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-block timings of the other workload shapes")
     ap.add_argument("--mx", action="store_true",
                     help="with --only qkv/out_proj/ffn1/ffn2: the MXFP8 linear")
     return ap.parse_args()
@@ -425,6 +432,61 @@ def run_only(args):
     return 0
 
 
+def block_timings(dh: int) -> dict:
+    """ms per block (block_forward, mod computed from t) at the other workload
+    shapes: the small block, the 2048^2 and 4096^2 canvases and the edit
+    request with four references; random device weights, median of 5."""
+    import torch
+
+    from image_generation_b200 import h3dit as Hb
+    from image_generation_b200 import synth
+
+    out = {}
+    names = ["small_block", "block_2k", "block_4k", "edit_4ref"]
+    if dh == 128:
+        names = ["block_2k_dh128", "block_4k_dh128", "edit_4ref_dh128"]
+    for name in names:
+        w = synth.WORKLOADS[name]
+        d = w.dims
+        I = d.heads * d.head_dim
+        g = torch.Generator(device="cuda")
+        g.manual_seed(7)
+        r = lambda *shape: (torch.randn(*shape, device="cuda", generator=g) * 0.02).bfloat16()
+        tw = {"w_t1": torch.randn(d.hidden, 256, device="cuda", generator=g) * 0.02,
+              "b_t1": torch.zeros(d.hidden, device="cuda"),
+              "w_t2": torch.randn(d.hidden, d.hidden, device="cuda", generator=g) * 0.02,
+              "b_t2": torch.zeros(d.hidden, device="cuda")}
+        blk = {"w_qkv": r(3 * I, d.hidden), "w_o": r(d.hidden, I), "w_ff1": r(d.ffn, d.hidden),
+               "w_ff2": r(d.hidden, d.ffn), "w_ada": r(6 * d.hidden, d.hidden),
+               "b_ada": torch.zeros(6 * d.hidden, device="cuda")}
+        ctx = Hb.Context(Hb.make_config(d.hidden, d.heads, d.head_dim, d.ffn, 1, w.n_tokens), tw, [blk])
+        n_img = w.n_tokens - w.n_txt
+        x_txt = torch.randn(w.n_txt, d.hidden, device="cuda", generator=g).bfloat16()
+        x_img = torch.randn(n_img, d.hidden, device="cuda", generator=g).bfloat16()
+        grids = list(w.grids)
+        for _ in range(2):
+            ctx.block_forward(0, 0.5, x_img, grids, x_txt)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        ev[0].record()
+        for i in range(5):
+            ctx.block_forward(0, 0.5, x_img, grids, x_txt)
+            ev[i + 1].record()
+        torch.cuda.synchronize()
+        if ctx.sync_status() != 0:
+            raise RuntimeError(f"block timing failed for {name}")
+        ms = sorted(ev[i].elapsed_time(ev[i + 1]) for i in range(5))
+        out[name] = {"ms": round(ms[2], 3), "tokens": w.n_tokens,
+                     "tflops": round(block_flops(w.n_tokens, d) / ms[2] / 1e9, 1)}
+        ctx.close()
+        del blk, tw
+    return out
+
+
+def block_flops(n: int, d) -> float:
+    I = d.heads * d.head_dim
+    return 8.0 * n * d.hidden * I + 4.0 * n * d.hidden * d.ffn + 4.0 * n * n * I
+
+
 def run_h3dit(args):
     import torch
 
@@ -463,9 +525,12 @@ def run_h3dit(args):
     barrier()
     ctx.profile_begin()
     n0 = ctx.launch_count()
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps - 1)]
     e0.record(stream)
     for i in range(args.steps):
         ctx.step(ts[args.warmup + i], x_img, grids, x_txt)
+        if i + 1 < args.steps:
+            marks[i].record(stream)
     e1.record(stream)
     barrier()
     launches = ctx.launch_count() - n0
@@ -476,6 +541,26 @@ def run_h3dit(args):
     if st != 0:
         raise RuntimeError(f"timed steps failed with status {st}")
     ms_step = elapsed / args.steps
+    bounds = [e0] + marks + [e1]
+    per_step = sorted(bounds[i].elapsed_time(bounds[i + 1]) for i in range(args.steps))
+
+    # the same step replayed from a CUDA graph (launch overhead removed)
+    graph_ms = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            ctx.step(ts[0], x_img, grids, x_txt)
+        graph.replay()
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+        barrier()
+        graph_ms = slowest_rank(e0.elapsed_time(e1), dist) / args.steps
+        del graph
+        if ctx.sync_status() != 0:
+            raise RuntimeError("graph-replayed steps failed")
 
     # end to end: host (pinned) tokens in, step, tokens back to the host
     e2e = None
@@ -556,7 +641,19 @@ def run_h3dit(args):
                                             float(peaks["bf16_tflops_sustained"]), 4),
             "roofline": roof, "kernels": kernels, "gpu_launches": launches,
             "e2e": e2e, "clocks": clk,
+            "step_ms": {"median": round(per_step[len(per_step) // 2], 2),
+                        "min": round(per_step[0], 2), "max": round(per_step[-1], 2)},
+            "six_step_ms": round(6 * ms_step, 1),
+            "graph_ms_per_step": None if graph_ms is None else round(graph_ms, 2),
         }
+        gemm_kinds = ("qkv", "out_proj", "ffn1", "ffn2")
+        if all(prof[k][1] for k in gemm_kinds):
+            g_ms = sum(prof[k][0] for k in gemm_kinds)
+            g_fl = sum(flops_per_launch(k, N_TOK, dh) * prof[k][1] for k in gemm_kinds)
+            line["gemm_tflops"] = round(g_fl / g_ms / 1e9, 1)
+            line["attention_tflops"] = kernels.get("attention", {}).get("tflops")
+        if world == 1 and not args.no_configs:
+            line["ms_per_block"] = block_timings(dh)
         if world == 1 and not args.no_cpu_baseline:
             v, desc, threads, secs = oracle_sample(dh)
             line["cpu_baseline"] = {"value": round(v, 1), "unit": "ms", "cores": threads,
