@@ -5,6 +5,7 @@
     python bench.py [--gpus N --steps K --warmup W] [--head-dim 96|128]
     python bench.py --impl reference          # the CPU oracle on a bounded sample
     python bench.py --only attention          # one kernel kind alone (for profilers)
+    python bench.py --oracle-configs          # the CPU oracle on every workload shape
 
 Rank 0 prints one JSON line. Besides the contract's keys it carries the
 per-step median/min/max, the same step replayed from a CUDA graph, the 6-step
@@ -53,6 +54,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-mxfp8", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the graph-replayed step timing")
+    ap.add_argument("--oracle-configs", action="store_true",
+                    help="time the CPU oracle on every workload shape (minutes) and exit")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the per-block timings of the other workload shapes")
     ap.add_argument("--mx", action="store_true",
@@ -291,6 +294,54 @@ def oracle_sample(dh: int, rows_a: int = 32, rows_b: int = 544, seed: int = 0):
             f"extrapolated linearly to {N_TOK} rows and x{L} blocks, plus the timestep MLP "
             f"({t_time * 1e3:.1f} ms) and {L} AdaLN projections ({t_ada * 1e3:.1f} ms each)")
     return step_ms, desc, threads, sum(times) + t_time + t_ada
+
+
+def run_oracle_configs(args):
+    """The oracle (float64 numpy) timed on this host: the small block and the
+    2048^2 block in full, the 4096^2 block and the edit request by sampled
+    query rows extrapolated linearly (labelled), and the 50-block step from
+    the 4096^2 block. One JSON line; test infrastructure, not a bench value."""
+    import numpy as np
+
+    from image_generation_b200 import synth
+    from oracle import dit_block as O
+
+    dh = args.head_dim
+    out = {}
+    for name in ("small_block", "block_2k", "block_4k", "edit_4ref"):
+        w = synth.WORKLOADS[name if dh == 96 or name == "small_block" else name + "_dh128"]
+        d = w.dims
+        cfg = O.config_for(d.hidden, d.heads, d.head_dim, d.ffn)
+        bw = synth.block_weights(d, w.seed)
+        tw = synth.time_weights(d, w.seed)
+        inp = synth.workload_inputs(w)
+        x = O.pack(inp["x_txt"], inp["x_img"])
+        pos = O.token_positions(w.n_txt, w.grids)
+        mod = O.adaln_modulation(O.timestep_condition(inp["t"], tw, cfg), bw["w_ada"], bw["b_ada"])
+        if w.n_tokens <= 5000:
+            t0 = time.perf_counter()
+            O.block_forward(x, mod, bw, pos, cfg)
+            out[name] = {"s_per_block": round(time.perf_counter() - t0, 2), "tokens": w.n_tokens,
+                         "how": "full block"}
+        else:
+            rng = np.random.default_rng(0)
+            O.block_forward(x, mod, bw, pos, cfg, rows=np.arange(8))  # untimed: first-touch costs
+            t = []
+            for r in (32, 544):
+                rows = np.sort(rng.choice(w.n_tokens, r, replace=False))
+                t0 = time.perf_counter()
+                O.block_forward(x, mod, bw, pos, cfg, rows=rows)
+                t.append(time.perf_counter() - t0)
+            slope = max((t[1] - t[0]) / 512, 0.0)
+            est = max(t[0] - 32 * slope, 0.0) + slope * w.n_tokens
+            out[name] = {"s_per_block": round(est, 1), "tokens": w.n_tokens,
+                         "how": f"extrapolated from 32 and 544 query rows ({t[0]:.1f} s, {t[1]:.1f} s)"}
+    blk = out["block_4k"]["s_per_block"]
+    out["step_4k"] = {"s_per_step": round(L * blk, 0), "how": f"extrapolated: {L} x the 4096^2 block"}
+    out["six_steps_4k"] = {"s": round(6 * L * blk, 0), "how": "extrapolated: 6 steps"}
+    print(json.dumps({"oracle_timing": out, "head_dim": dh, "cores": _blas_threads(),
+                      "dtype": "f64"}), flush=True)
+    return 0
 
 
 def _blas_threads() -> int:
@@ -697,6 +748,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.oracle_configs:
+        return run_oracle_configs(args)
     if args.only:
         return run_only(args)
     return run_h3dit(args)
