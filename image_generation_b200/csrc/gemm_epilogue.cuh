@@ -27,12 +27,31 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
   tn = local / gm;
 }
 
+// erf(z) for z >= 0 by Abramowitz & Stegun, Handbook of Mathematical
+// Functions, 7.1.26: 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) e^(-z^2)
+// with t = 1 / (1 + p z), |error| <= 1.5e-7 (far below the bf16 or E4M3
+// rounding of the GELU output). Two MUFU operations (reciprocal, 2^x) and a
+// handful of FMAs per element, which keeps the FFN1 epilogue cheap.
+__device__ __forceinline__ float erf_nonneg(float z) {
+  float t;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(0.3275911f, z, 1.0f)));
+  float poly = fmaf(1.061405429f, t, -1.453152027f);
+  poly = fmaf(poly, t, 1.421413741f);
+  poly = fmaf(poly, t, -0.284496736f);
+  poly = fmaf(poly, t, 0.254829592f);
+  poly *= t;
+  const float e = ex2_approx(-(z * z) * 1.4426950408889634f);  // e^(-z^2)
+  return fmaf(-poly, e, 1.0f);
+}
+
 __device__ __forceinline__ float gelu_f(float x, int tanh_form) {
   if (tanh_form) {
     const float u = 0.7978845608028654f * (x + 0.044715f * x * x * x);
     return 0.5f * x * (1.0f + tanhf(u));
   }
-  return 0.5f * x * (1.0f + erff(x * 0.7071067811865476f));
+  // x Phi(x) = x (1 + erf(x / sqrt 2)) / 2, erf odd
+  const float er = copysignf(erf_nonneg(fabsf(x) * 0.7071067811865476f), x);
+  return x * fmaf(0.5f, er, 0.5f);
 }
 
 // Store `W` consecutive fp32 values as bf16 (W multiple of 8, 16-byte aligned).
