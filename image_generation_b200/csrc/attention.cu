@@ -35,9 +35,9 @@ namespace h3 {
 namespace {
 
 constexpr int BQ = kAttnBQ;                  // rows of one query tile
-constexpr int BKV = kAttnBKV;                // keys per KV tile
-constexpr int SBUF = BKV == 64 ? 2 : 1;      // S buffers per query tile (128 columns each tile)
-constexpr int NS = BKV == 64 ? 4 : 2;        // K/V ring stages (128 KiB)
+constexpr int BKV = kAttnBKV;                // keys per KV tile (64)
+constexpr int SBUF = 2;                      // S buffers per query tile (128 columns each tile)
+constexpr int NS = 4;                        // K/V ring stages (128 KiB)
 constexpr uint32_t QBOX = 128 * 128;         // one [128 rows x 64 bf16] swizzled box
 constexpr uint32_t KBOX = BKV * 128;         // one [64 rows x 64 bf16] swizzled box
 constexpr uint32_t Q_BYTES = 2 * QBOX;       // one query tile (d_h <= 128)
@@ -52,50 +52,6 @@ constexpr int NUM_BARS = 1 + 2 * NS + 4 + 4 + 2 + 2 + 2;
 constexpr int SMEM_BYTES = 2 * Q_BYTES + NS * STAGE_BYTES + 1024 + NUM_BARS * 8 + 16;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;    // log2 units
-
-// Share of the exponentials computed on the FMA pipe instead of the MUFU
-// pipe: 0 none, 1 one pair in four, 2 one pair in two. On paper the MUFU
-// work per KV tile at head_dim 96 (2 x 128 x 128 ex2 at 16 per clock per SM)
-// exceeds the tensor work, but measured on B200 the extra FMA-pipe work costs
-// more than it saves at both head dims, so the default is none.
-#ifdef H3_EXP_EMU
-template <int DH>
-constexpr int kExpEmu = H3_EXP_EMU;
-#else
-template <int DH>
-constexpr int kExpEmu = 0;
-#endif
-
-// 2^x for x <= 126 on the FMA pipe, two lanes at a time (Cody-Waite
-// split): x = n + f with n = round(x) from the 1.5 * 2^23 rounding trick and
-// |f| <= 1/2; 2^f from a degree-3 polynomial, minimax in relative error on
-// [-1/2, 1/2] (Remez exchange, max relative error 7.5e-5, well below the 2^-9
-// rounding of bf16 P); 2^n is added into the exponent field. Inputs below
-// -126 (masked scores are -inf) clamp to about 2^-126.
-H3_DEV uint64_t exp2_poly2(uint64_t x2) {
-  float x0, x1;
-  f2_unpack(x2, x0, x1);
-  x2 = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-  const uint64_t t2 = f2_add(x2, f2_pack(12582912.0f, 12582912.0f));
-  const uint64_t nf2 = f2_add(t2, f2_pack(-12582912.0f, -12582912.0f));  // round(x)
-  float n0, n1;
-  f2_unpack(nf2, n0, n1);
-  const uint64_t f2 = f2_add(x2, f2_pack(-n0, -n1));  // x - round(x)
-  uint64_t q2 = f2_fma(f2_pack(0.0551716685f, 0.0551716685f), f2,
-                       f2_pack(0.2426111251f, 0.2426111251f));
-  q2 = f2_fma(q2, f2, f2_pack(0.6932609677f, 0.6932609677f));
-  q2 = f2_fma(q2, f2, f2_pack(0.9999280572f, 0.9999280572f));
-  float q0, q1, t0, t1;
-  f2_unpack(q2, q0, q1);
-  f2_unpack(t2, t0, t1);
-  return f2_pack(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
-                 __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
-}
-
-template <int EMU>
-H3_DEV constexpr bool use_poly(int pair) {
-  return EMU == 1 ? (pair % 4) == 3 : EMU == 2 ? (pair % 2) == 1 : false;
-}
 
 // One row's scores for 64 keys from TMEM; keys at or past `valid` are -inf
 // (only the last KV tile has any).
@@ -127,7 +83,6 @@ H3_DEV float row_max64(const float (&s)[64]) {
 
 // p_i = 2^(s_i * scale_log2 - m) for 64 scores, two at a time: added into the
 // four partial row sums and packed as bf16 pairs (the A operand of PV).
-template <int DH>
 H3_DEV void exp_pack64(const float (&s)[64], float sl2, float m, uint64_t (&part)[4],
                        uint32_t (&pk)[32]) {
   const uint64_t sl2x2 = f2_pack(sl2, sl2);
@@ -135,14 +90,9 @@ H3_DEV void exp_pack64(const float (&s)[64], float sl2, float m, uint64_t (&part
 #pragma unroll
   for (int i = 0; i < 64; i += 2) {
     const uint64_t y2 = f2_fma(f2_pack(s[i], s[i + 1]), sl2x2, negm2);
-    uint64_t e2;
-    if (use_poly<kExpEmu<DH>>(i / 2)) {
-      e2 = exp2_poly2(y2);
-    } else {
-      float y0, y1;
-      f2_unpack(y2, y0, y1);
-      e2 = f2_pack(ex2_approx(y0), ex2_approx(y1));
-    }
+    float y0, y1;
+    f2_unpack(y2, y0, y1);
+    const uint64_t e2 = f2_pack(ex2_approx(y0), ex2_approx(y1));
     part[(i / 2) & 3] = f2_add(part[(i / 2) & 3], e2);
     float e0, e1;
     f2_unpack(e2, e0, e1);
@@ -285,10 +235,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t v_src = sKV + (j % NS) * STAGE_BYTES + KV_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk) {
-          // A: P_t(j) in TMEM, 16 keys = 8 packed columns per step (with
-          // 128 keys, keys 64..127 sit in columns 64..95)
-          const uint32_t p_col = 8 * kk + (kk >= 4 ? 32 : 0);
-          umma_bf16_ts(o_tmem, s_base + static_cast<uint32_t>(BKV * (j % SBUF)) + p_col,
+          // A: P_t(j) in TMEM, 16 keys = 8 packed columns per step
+          umma_bf16_ts(o_tmem, s_base + static_cast<uint32_t>(BKV * (j % SBUF)) + 8 * kk,
                        desc_sw128(v_src + kk * 16 * 128, KBOX, 1024), IDESC_O,
                        (j > 0 || kk > 0) ? 1u : 0u);
         }
@@ -336,38 +284,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       };
       uint64_t part[4] = {0, 0, 0, 0};
-      if constexpr (BKV == 64) {
+      {
         float sc[64];
         load_scores64(tS, sc, valid);
         update_max(row_max64(sc));
         uint32_t pk[32];
-        exp_pack64<DH>(sc, sl2, m, part, pk);
+        exp_pack64(sc, sl2, m, part, pk);
         tmem_st32(tS, pk);
-      } else {
-        // 128 keys in two halves of 64 columns, read twice from TMEM (a
-        // second read is cheaper than holding 128 scores in registers): the
-        // max over both halves, then each half's P over its own scores, keys
-        // 64..127 to columns 64..95 first, then keys 0..63 to columns 0..31.
-        float mx_lo;
-        {
-          float lo[64];
-          load_scores64(tS, lo, valid);
-          mx_lo = row_max64(lo);
-        }
-        asm volatile("" : "+f"(mx_lo));  // the first half is reduced before the second loads
-        {
-          float hi[64];
-          load_scores64(tS + 64, hi, valid - 64);
-          update_max(fmaxf(mx_lo, row_max64(hi)));
-        }
-#pragma unroll 1
-        for (int h = 64; h >= 0; h -= 64) {
-          float sc[64];
-          load_scores64(tS + h, sc, valid - h);
-          uint32_t pk[32];
-          exp_pack64<DH>(sc, sl2, m, part, pk);
-          tmem_st32(tS + h, pk);
-        }
       }
       float sum;
       {

@@ -75,13 +75,10 @@ cudaError_t launch_gemm_pair(const CUtensorMap &a, const CUtensorMap &b, const G
 // Clusters of the paired kernel that fit on the device at once (0: unusable).
 int gemm_pair_max_clusters(int epilogue);
 
-// Attention tiles: 128 queries per query tile (two per CTA), kAttnBKV keys per
-// KV tile (64: two S buffers per query tile in TMEM; 128: one).
-#ifndef H3_ATTN_BKV
-#define H3_ATTN_BKV 64
-#endif
+// Attention tiles: 128 queries per query tile (two per CTA), 64 keys per KV
+// tile (two S buffers per query tile in TMEM).
 constexpr int kAttnBQ = 128;
-constexpr int kAttnBKV = H3_ATTN_BKV;
+constexpr int kAttnBKV = 64;
 cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
                              const AttnParams &p, int head_dim, int heads, bool out_mx,
                              cudaStream_t s);
