@@ -20,7 +20,7 @@
  *   - Matrices are row-major. Weights use the nn.Linear layout [out, in].
  *   - All work is enqueued on `cuda_stream` (a cudaStream_t; NULL is the
  *     legacy default stream) and is asynchronous. No call synchronises except
- *     h3dit_sync_status. Calls never abort or exit the process.
+ *     h3dit_sync_status (and h3dit_create, once, before it returns). Calls never abort or exit the process.
  *   - A context is used from one host thread at a time; two calls on one
  *     context must not overlap on the GPU (they share its workspace).
  *   - On an error, nothing is enqueued (validation happens first) unless the
@@ -107,14 +107,19 @@ const char *h3dit_last_error(const h3dit_ctx *ctx);
 /* Bytes of device workspace h3dit_create needs for `cfg`, or 0 if `cfg` is
  * invalid. It covers the fp32 residual stream, the bf16 activations (xm,
  * Q|K|V, attention output, FFN hidden), the per-step modulation table
- * [n_blocks][6][D], the timestep vectors, the RoPE table and a status word. */
+ * [n_blocks][6][D], the timestep vectors, the RoPE table and a status word;
+ * with H3DIT_PRECISION_MXFP8 also the MXFP8 activations and their scales and
+ * every block's quantized linears (E4M3 weights, their scales, and the
+ * scales repacked for 224-column tiles where N is a multiple of 224). */
 size_t h3dit_workspace_bytes(const h3dit_config *cfg);
 
 /* Create a context. `blocks` points to cfg->n_blocks host structs whose device
  * pointers must stay valid until h3dit_destroy. `workspace` is device memory of
  * at least h3dit_workspace_bytes(cfg) bytes, 256-byte aligned, lent to the
- * context for its life. Enqueues a small copy of the weight pointer table on
- * `cuda_stream`. On error *out is set to NULL. */
+ * context for its life. Copies the weight pointer table to the device and,
+ * with H3DIT_PRECISION_MXFP8, quantizes every block's linears, on
+ * `cuda_stream`, then synchronises that stream once before returning (the
+ * host-side table must have been consumed). On error *out is set to NULL. */
 h3dit_status h3dit_create(const h3dit_config *cfg, const h3dit_time_weights *time_w,
                           const h3dit_block_weights *blocks, void *workspace, size_t ws_bytes,
                           void *cuda_stream, h3dit_ctx **out);
