@@ -20,7 +20,8 @@
  *   - Matrices are row-major. Weights use the nn.Linear layout [out, in].
  *   - All work is enqueued on `cuda_stream` (a cudaStream_t; NULL is the
  *     legacy default stream) and is asynchronous. No call synchronises except
- *     h3dit_sync_status (and h3dit_create, once, before it returns). Calls never abort or exit the process.
+ *     h3dit_sync_status (and h3dit_create, once, before it returns). Calls
+ *     never abort or exit the process.
  *   - A context is used from one host thread at a time; two calls on one
  *     context must not overlap on the GPU (they share its workspace).
  *   - On an error, nothing is enqueued (validation happens first) unless the
