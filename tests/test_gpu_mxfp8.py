@@ -275,14 +275,24 @@ def test_block_linear_mx_stages(dims):
     """Each of a block's MXFP8 linears through the stage entry point, on the
     context's own quantized weights: wide (128 x 224) tiles where every N is
     a multiple of 224 (hidden 2688), the 128-wide kernel otherwise."""
+    _block_linear_mx_stages(dims, [(0, 11, 19)], 9)
+
+
+def test_block_linear_mx_wide_several_tiles_per_cta():
+    """Hidden 2688, 1065 tokens: 9 row tiles of 128 (the last ragged) x 36
+    QKV (16 FFN1, 12 out / FFN2) column tiles of 224, so with 148 CTAs each
+    takes two or three tiles and both TMEM accumulators turn over."""
+    _block_linear_mx_stages(synth.Dims(2688, 28, 96, 3584), [(0, 32, 33)], 9)
+
+
+def _block_linear_mx_stages(dims, grids, n_txt):
     from image_generation_b200 import h3dit as H
 
-    ctx, _, bws = _ctx(dims, max_tokens=300, precision=1)
+    pos = O.token_positions(n_txt, grids)
+    ctx, _, bws = _ctx(dims, max_tokens=max(300, pos.shape[0]), precision=1)
     ocfg = O.config_for(dims.hidden, dims.heads, dims.head_dim, dims.ffn)
     I, D, F = ocfg.inner, dims.hidden, dims.ffn
     bw = bws[0]
-    grids, n_txt = [(0, 11, 19)], 9
-    pos = O.token_positions(n_txt, grids)
     m = pos.shape[0]
     # QKV + RoPE
     x = synth.tokens(m, D, 21, "x")
