@@ -40,7 +40,8 @@ Readings where the pages are silent (each listed in the design notes):
   reference image k is frame k; attention is bidirectional, unmasked, scaled
   by 1/sqrt(head_dim).
 
-Parity pins: tests/test_oracle_pins.py. The real model's numbers are "parity
+Parity pins: tests/test_oracle_pins.py, and tests/test_oracle_c.py against the
+independent C oracle (oracle/h3ref.c). The real model's numbers are "parity
 unpinned" (no trained weights or printed activations exist to compare with).
 """
 from __future__ import annotations
