@@ -1,7 +1,8 @@
 // C ABI of libh3dit (declared in include/h3dit.h): argument checks, the
 // workspace plan, TMA tensor-map encoding and the order of kernel launches
 // for one DiT block and one sampling step. All compute runs in the kernels of
-// gemm.cu, attention.cu and elementwise.cu; this file only marshals.
+// gemm.cu, gemm_pair.cu, gemm_mx.cu, attention.cu and elementwise.cu; this
+// file only marshals.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -224,7 +225,13 @@ struct Launch {
     }
   }
   ~Launch() {
-    if (on && cudaEventRecord(rec.end, s) == cudaSuccess) ctx->records.push_back(rec);
+    if (on && cudaEventRecord(rec.end, s) == cudaSuccess) {
+      ctx->records.push_back(rec);
+      return;
+    }
+    // not recorded: the events go back to the pool
+    if (rec.begin) ctx->event_pool.push_back(rec.begin);
+    if (rec.end) ctx->event_pool.push_back(rec.end);
   }
 };
 }  // namespace
