@@ -381,6 +381,94 @@ def block_forward_mx(x, mod, w: Dict[str, np.ndarray], pos: np.ndarray, cfg: Blo
     return xr + g2 * linear_mx(u, w["w_ff2"])
 
 
+# --- Around the block loop: patchify, embeddings, output layer, sampler ------
+# [card] "Model Architecture": the image VAE has 16x spatial downsampling and
+# 24 latent channels; the DiT patchifies the latent with a 2x2 patch (so one
+# token covers 32x32 pixels); the embedding, timestep and output layers are
+# FP32. The real per-step output heads and the sampling schedule ship in a
+# file these pages do not give, so the plain reading stands in for them: a
+# DiT final layer (RMSNorm, AdaLN shift/scale from the timestep condition,
+# Linear D -> 96 with bias) predicting the flow velocity dz/dt, and Euler
+# steps from t = 1 (noise) to t = 0 over the step_forward schedule.
+
+LATENT_CHANNELS = 24
+PATCH = 2
+
+
+def patchify(z, patch: int = PATCH) -> np.ndarray:
+    """Latent z [C, Hl, Wl] -> tokens [(Hl/p) (Wl/p), C p p]. Token (r, c) is
+    row-major over the (Hl/p, Wl/p) grid, the order token_positions gives an
+    image; feature ch * p^2 + i * p + j holds latent pixel (p r + i, p c + j)
+    of channel ch."""
+    z = _f64(z)
+    C, Hl, Wl = z.shape
+    if Hl % patch or Wl % patch:
+        raise ValueError("latent sides must be multiples of the patch")
+    h, w = Hl // patch, Wl // patch
+    t = z.reshape(C, h, patch, w, patch)          # ch, r, i, c, j
+    return t.transpose(1, 3, 0, 2, 4).reshape(h * w, C * patch * patch)
+
+
+def unpatchify(tokens, channels: int, h: int, w: int, patch: int = PATCH) -> np.ndarray:
+    """The inverse of patchify: tokens [h w, C p p] -> latent [C, h p, w p]."""
+    t = _f64(tokens).reshape(h, w, channels, patch, patch)   # r, c, ch, i, j
+    return t.transpose(2, 0, 3, 1, 4).reshape(channels, h * patch, w * patch)
+
+
+def patch_embed(tokens, w, b) -> np.ndarray:
+    """FP32 patch embedding ([card]): tokens [n, C p p] W^T + b -> [n, D]."""
+    return _f64(tokens) @ _f64(w).T + _f64(b)
+
+
+def final_layer(x, c, w_mod, b_mod, w_out, b_out, eps: float) -> np.ndarray:
+    """Output layer on the image tokens x [n, D]: [shift, scale] =
+    W_mod SiLU(c) + b_mod (W_mod [2D, D]), then
+    (RMSNorm(x) (1 + scale) + shift) W_out^T + b_out (W_out [C p p, D])."""
+    shift, scale = (_f64(w_mod) @ silu(c) + _f64(b_mod)).reshape(2, -1)
+    return norm_modulate(x, shift, scale, eps) @ _f64(w_out).T + _f64(b_out)
+
+
+def sampling_timesteps(n_steps: int) -> np.ndarray:
+    """t_k = 1 - k / n for k = 0 .. n: the n network evaluations happen at
+    t_0 .. t_{n-1}, and the last Euler step lands on t_n = 0."""
+    return 1.0 - np.arange(n_steps + 1, dtype=np.float64) / n_steps
+
+
+def euler_update(z, v, t: float, t_next: float) -> np.ndarray:
+    """One step of dz/dt = v: z(t_next) = z(t) + (t_next - t) v."""
+    return _f64(z) + (float(t_next) - float(t)) * _f64(v)
+
+
+def dit_velocity(z, x_txt, t: float, tw: Dict[str, np.ndarray],
+                 blocks: Sequence[Dict[str, np.ndarray]], io: Dict[str, np.ndarray],
+                 cfg: BlockConfig) -> np.ndarray:
+    """The denoiser on one target latent z [C, Hl, Wl] with text tokens
+    x_txt [n_txt, D]: patchify, embed, the packed step through every block,
+    the output layer on the image tokens, unpatchify. io holds w_in [D, 96],
+    b_in [D], w_mod [2D, D], b_mod [2D], w_out [96, D], b_out [96]."""
+    C, Hl, Wl = _f64(z).shape
+    h, w = Hl // PATCH, Wl // PATCH
+    x_img = patch_embed(patchify(z), io["w_in"], io["b_in"])
+    n_txt = _f64(x_txt).shape[0]
+    pos = token_positions(n_txt, [(0, h, w)])
+    y = step_forward(pack(x_txt, x_img), t, tw, blocks, pos, cfg)
+    c = timestep_condition(t, tw, cfg)
+    out = final_layer(y[n_txt:], c, io["w_mod"], io["b_mod"], io["w_out"], io["b_out"],
+                      cfg.norm_eps)
+    return unpatchify(out, C, h, w)
+
+
+def denoise(z_noise, velocity, n_steps: int) -> np.ndarray:
+    """Euler integration of dz/dt = velocity(z, t) from t = 1 to t = 0 over
+    sampling_timesteps(n_steps); velocity is any callable (the DiT above, or a
+    closed-form field in the tests)."""
+    ts = sampling_timesteps(n_steps)
+    z = _f64(z_noise)
+    for k in range(n_steps):
+        z = euler_update(z, velocity(z, ts[k]), ts[k], ts[k + 1])
+    return z
+
+
 def block_flops(n: int, hidden: int, inner: int, ffn: int) -> int:
     """Algorithmic flops of one block: QKV 6NDI, out-proj 2NDI, FFN 4NDF,
     attention 4N^2 I (QK^T and PV over all N^2 pairs, no causal halving)."""
