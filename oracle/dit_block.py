@@ -38,7 +38,10 @@ Readings where the pages are silent (each listed in the design notes):
   each a rotate-half 1-D RoPE over its own contiguous 2*s channels with
   frequencies theta^(-j/s), theta 10000; text tokens sit at position (0,0,0);
   reference image k is frame k; attention is bidirectional, unmasked, scaled
-  by 1/sqrt(head_dim).
+  by 1/sqrt(head_dim). Around the block loop: 2x2 patches of the 24-channel
+  latent in pixel-unshuffle order, an FP32 Linear(96 -> D) embedding with
+  bias, a DiT output layer (RMSNorm, AdaLN shift/scale, Linear(D -> 96) with
+  bias) predicting the flow velocity, and Euler steps from t = 1 to t = 0.
 
 Parity pins: tests/test_oracle_pins.py, and tests/test_oracle_c.py against the
 independent C oracle (oracle/h3ref.c). The real model's numbers are "parity
