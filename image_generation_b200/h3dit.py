@@ -164,8 +164,20 @@ def grids_array(grids: Sequence[Tuple[int, int, int]]):
 
 # ---------------------------------------------------------------- torch helpers
 
-def _ptr(t) -> int | None:
-    return None if t is None else t.data_ptr()
+def _ptr(t, dense: bool = True) -> int | None:
+    """Device address of a tensor argument. Every tensor must be on a CUDA
+    device. Those the ABI reads as dense arrays must be contiguous; the
+    attention operands are strided row views (their row stride is passed
+    separately) and only need a unit stride along the last axis."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise H3DitError(H3DIT_ERR_INVALID_ARG, "tensor argument is not on a CUDA device")
+    if dense and not t.is_contiguous():
+        raise H3DitError(H3DIT_ERR_INVALID_ARG, "tensor argument is not contiguous")
+    if not dense and t.dim() > 0 and t.stride(-1) != 1:
+        raise H3DitError(H3DIT_ERR_INVALID_ARG, "strided operand needs unit stride in its last axis")
+    return t.data_ptr()
 
 
 def _stream(stream=None) -> int:
@@ -236,8 +248,9 @@ class Context:
                                      _ptr(gate), _ptr(rope_table), _stream(stream)))
 
     def attention(self, q, k, v, ld_qkv: int, o, ld_o: int, n: int, stream=None) -> None:
-        self._check(lib.h3dit_attention(self.handle, _ptr(q), _ptr(k), _ptr(v), ld_qkv, _ptr(o),
-                                        ld_o, n, _stream(stream)))
+        self._check(lib.h3dit_attention(self.handle, _ptr(q, False), _ptr(k, False),
+                                        _ptr(v, False), ld_qkv, _ptr(o, False), ld_o, n,
+                                        _stream(stream)))
 
     def block_forward(self, block: int, t: float, x_img, grids, x_txt, mod=None,
                       stream=None) -> None:
@@ -271,8 +284,9 @@ class Context:
                                                   _stream(stream)))
 
     def attention_mx(self, q, k, v, ld_qkv: int, o, o_sf, n: int, stream=None) -> None:
-        self._check(lib.h3dit_attention_mx(self.handle, _ptr(q), _ptr(k), _ptr(v), ld_qkv,
-                                           _ptr(o), _ptr(o_sf), n, _stream(stream)))
+        self._check(lib.h3dit_attention_mx(self.handle, _ptr(q, False), _ptr(k, False),
+                                           _ptr(v, False), ld_qkv, _ptr(o), _ptr(o_sf), n,
+                                           _stream(stream)))
 
     def selftest_bounded_wait(self, limit_us: int, stream=None) -> None:
         self._check(lib.h3dit_selftest_bounded_wait(self.handle, limit_us, _stream(stream)))

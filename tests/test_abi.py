@@ -128,3 +128,15 @@ def test_mx_scale_layout_size():
     rows, k = 256, 384
     offs = {H.mx_sf_offset(r, s, k) for r in range(rows) for s in range(k // 32)}
     assert len(offs) == rows * k // 32 and max(offs) < H.mx_scale_bytes(rows, k)
+
+
+def test_binding_rejects_host_tensors_before_the_library_sees_them():
+    """Tensor arguments go to the kernels as device addresses, so a host tensor
+    is refused in the binding (the library cannot tell a host address apart)."""
+    import torch
+
+    assert H._ptr(None) is None
+    for dense in (True, False):
+        with pytest.raises(H.H3DitError) as e:
+            H._ptr(torch.zeros(4), dense)
+        assert e.value.status == H.H3DIT_ERR_INVALID_ARG
