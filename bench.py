@@ -300,7 +300,8 @@ def run_oracle_configs(args):
     """The oracle (float64 numpy) timed on this host: the small block and the
     2048^2 block in full, the 4096^2 block and the edit request by sampled
     query rows extrapolated linearly (labelled), and the 50-block step from
-    the 4096^2 block. One JSON line; test infrastructure, not a bench value."""
+    the 4096^2 block; plus the C oracle's plain-fp32 build on the small block.
+    One JSON line; test infrastructure, not a bench value."""
     import numpy as np
 
     from image_generation_b200 import synth
@@ -339,6 +340,27 @@ def run_oracle_configs(args):
     blk = out["block_4k"]["s_per_block"]
     out["step_4k"] = {"s_per_step": round(L * blk, 0), "how": f"extrapolated: {L} x the 4096^2 block"}
     out["six_steps_4k"] = {"s": round(6 * L * blk, 0), "how": "extrapolated: 6 steps"}
+    # the independent C oracle, plain fp32 loops on one core, on the small block
+    try:
+        from oracle import ref_c
+
+        ref = ref_c.load("f32")
+        w = synth.WORKLOADS["small_block"]
+        d = w.dims
+        cfg = O.config_for(d.hidden, d.heads, d.head_dim, d.ffn)
+        bw = synth.block_weights(d, w.seed)
+        inp = synth.workload_inputs(w)
+        x = O.pack(inp["x_txt"], inp["x_img"])
+        mod = O.adaln_modulation(O.timestep_condition(inp["t"], synth.time_weights(d, w.seed), cfg),
+                                 bw["w_ada"], bw["b_ada"])
+        pos = O.token_positions(w.n_txt, w.grids)
+        t0 = time.perf_counter()
+        ref.block_forward(x, mod, bw, pos, heads=d.heads, head_dim=d.head_dim,
+                          sections=cfg.rope_sections)
+        out["small_block_c_f32"] = {"s_per_block": round(time.perf_counter() - t0, 2),
+                                    "tokens": w.n_tokens, "how": "C oracle, fp32, 1 core"}
+    except (OSError, RuntimeError) as e:  # no C compiler on this host
+        out["small_block_c_f32"] = {"unavailable": str(e).splitlines()[0]}
     print(json.dumps({"oracle_timing": out, "head_dim": dh, "cores": _blas_threads(),
                       "dtype": "f64"}), flush=True)
     return 0
