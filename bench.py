@@ -39,6 +39,11 @@ N_TXT, GRID = 512, 128
 N_TOK = N_TXT + GRID * GRID
 METRIC = "ms per 50-block 4096^2 denoise step"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet dense tensor peaks (no 2:4 sparsity), for the fractions
+# reported beside the measured-peak ones.
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_FP8_TFLOPS = 4500.0
+C_LAT = 24  # latent channels (16x VAE, 24 channels; 2x2 patches of 96 features)
 
 
 def parse():
@@ -53,6 +58,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-mxfp8", action="store_true")
+    ap.add_argument("--no-denoise", action="store_true",
+                    help="skip the 6-step sampling loop timing (h3dit_denoise)")
     ap.add_argument("--no-graph", action="store_true", help="skip the graph-replayed step timing")
     ap.add_argument("--oracle-configs", action="store_true",
                     help="time the CPU oracle on every workload shape (minutes) and exit")
@@ -255,11 +262,13 @@ def timesteps(k: int):
 
 # ----------------------------------------------------------------- CPU oracle
 
-def oracle_sample(dh: int, rows_a: int = 32, rows_b: int = 544, seed: int = 0):
+def oracle_sample(dh: int, rows_a: int = 32, rows_b: int | None = 544, seed: int = 0):
     """Time the oracle on one block of the 4096^2 step for two query-row
     samples (keys and values always over all tokens) and extrapolate linearly
     to all rows and to the 50 blocks of a step, plus the per-step timestep MLP
-    and AdaLN projections. Returns (ms per step, description, threads)."""
+    and AdaLN projections: an estimate, not a timed step. Returns (ms per step,
+    description, threads, CPU seconds). With rows_b None only the first sample
+    runs (a warm-up) and the estimate is None."""
     import numpy as np
 
     from image_generation_b200 import synth
@@ -280,6 +289,8 @@ def oracle_sample(dh: int, rows_a: int = 32, rows_b: int = 544, seed: int = 0):
     t_ada = time.perf_counter() - t0
     times = []
     for r in (rows_a, rows_b):
+        if r is None:
+            return None, "", _blas_threads(), times[0]
         rows = np.sort(rng.choice(N_TOK, r, replace=False))
         t0 = time.perf_counter()
         O.block_forward(x, mod, w, pos, cfg, rows=rows)
@@ -289,11 +300,37 @@ def oracle_sample(dh: int, rows_a: int = 32, rows_b: int = 544, seed: int = 0):
     block_s = fixed + slope * N_TOK
     step_ms = 1e3 * (t_time + L * t_ada + L * block_s)
     threads = _blas_threads()
-    desc = (f"oracle (float64 numpy) on one block of the step for {rows_a} and {rows_b} query rows "
-            f"(K/V over all {N_TOK} tokens): {times[0]:.2f} s and {times[1]:.2f} s; "
+    desc = (f"estimate: oracle (float64 numpy) on one block of the step for {rows_a} and {rows_b} "
+            f"query rows (K/V over all {N_TOK} tokens): {times[0]:.2f} s and {times[1]:.2f} s; "
             f"extrapolated linearly to {N_TOK} rows and x{L} blocks, plus the timestep MLP "
             f"({t_time * 1e3:.1f} ms) and {L} AdaLN projections ({t_ada * 1e3:.1f} ms each)")
     return step_ms, desc, threads, sum(times) + t_time + t_ada
+
+
+def oracle_block_2k(dh: int, seed: int = 0):
+    """The oracle timed on one whole block of the 2048^2 workload (4608
+    tokens, every row): a measured CPU figure, not an extrapolation. Returns
+    (ms, description, threads)."""
+    import numpy as np
+
+    from image_generation_b200 import synth
+    from oracle import dit_block as O
+
+    w = synth.WORKLOADS["block_2k" if dh == 96 else "block_2k_dh128"]
+    d = w.dims
+    cfg = O.config_for(d.hidden, d.heads, d.head_dim, d.ffn)
+    bw = synth.block_weights(d, seed)
+    tw = synth.time_weights(d, seed)
+    inp = synth.workload_inputs(w)
+    x = O.pack(inp["x_txt"], inp["x_img"])
+    pos = O.token_positions(w.n_txt, w.grids)
+    t0 = time.perf_counter()
+    mod = O.adaln_modulation(O.timestep_condition(inp["t"], tw, cfg), bw["w_ada"], bw["b_ada"])
+    O.block_forward(x, mod, bw, pos, cfg)
+    ms = 1e3 * (time.perf_counter() - t0)
+    return ms, (f"oracle (float64 numpy), one whole 2048^2 block ({w.n_tokens} tokens, "
+                f"head_dim {d.head_dim}) with its timestep MLP and AdaLN projection, timed"), \
+        _blas_threads()
 
 
 def run_oracle_configs(args):
@@ -386,8 +423,8 @@ def run_reference(args):
         return 0
     vals = []
     desc, threads = "", 1
-    for _ in range(min(args.warmup, 1)):
-        oracle_sample(args.head_dim)
+    for _ in range(args.warmup):  # untimed: one short sample each
+        oracle_sample(args.head_dim, rows_a=8, rows_b=None)
     t_all = time.perf_counter()
     for _ in range(args.steps):
         v, desc, threads, _ = oracle_sample(args.head_dim)
@@ -396,14 +433,15 @@ def run_reference(args):
     value = sum(vals) / len(vals)
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "ms",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": min(args.warmup, 1),
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(value, 1), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, random-init weights)",
         "config": {"workload": workload_name(args.head_dim), "n_blocks": L, "tokens": N_TOK,
-                   "head_dim": args.head_dim, "parallelism": "replicas",
-                   "l2": "inputs larger than L2"},
+                   "head_dim": args.head_dim, "global_batch": world,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (~44 GB of weights read per step)"},
         "cpu_baseline": {"value": round(value, 1), "unit": "ms", "cores": threads,
-                         "kind": "oracle", "sample": desc},
+                         "kind": "oracle", "estimated": True, "sample": desc},
         "e2e": {"value": round(value, 1), "unit": "ms", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "wall_s": round(wall, 1),
@@ -507,8 +545,9 @@ def run_only(args):
 
 def block_timings(dh: int) -> dict:
     """ms per block (block_forward, mod computed from t) at the other workload
-    shapes: the small block, the 2048^2 and 4096^2 canvases and the edit
-    request with four references; random device weights, median of 5."""
+    shapes: the small block (head_dim 96 only), the 2048^2 and 4096^2 canvases
+    and the edit request with four references; random device weights, median
+    of 5, with the attention and GEMM rates from the library's events."""
     import torch
 
     from image_generation_b200 import h3dit as Hb
@@ -540,16 +579,25 @@ def block_timings(dh: int) -> dict:
         for _ in range(2):
             ctx.block_forward(0, 0.5, x_img, grids, x_txt)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        ctx.profile_begin()
         ev[0].record()
         for i in range(5):
             ctx.block_forward(0, 0.5, x_img, grids, x_txt)
             ev[i + 1].record()
         torch.cuda.synchronize()
+        prof = ctx.profile_end()
         if ctx.sync_status() != 0:
             raise RuntimeError(f"block timing failed for {name}")
         ms = sorted(ev[i].elapsed_time(ev[i + 1]) for i in range(5))
-        out[name] = {"ms": round(ms[2], 3), "tokens": w.n_tokens,
-                     "tflops": round(block_flops(w.n_tokens, d) / ms[2] / 1e9, 1)}
+        n = w.n_tokens
+        att_ms, att_cnt = prof["attention"]
+        gemm = ("qkv", "out_proj", "ffn1", "ffn2")
+        g_ms = sum(prof[k][0] for k in gemm)
+        g_fl = 5 * (8.0 * n * d.hidden * I + 4.0 * n * d.hidden * d.ffn)
+        out[name] = {"ms": round(ms[2], 3), "tokens": n, "head_dim": d.head_dim,
+                     "tflops": round(block_flops(n, d) / ms[2] / 1e9, 1),
+                     "attention_tflops": round(4.0 * n * n * I * att_cnt / att_ms / 1e9, 1),
+                     "gemm_tflops": round(g_fl / g_ms / 1e9, 1)}
         ctx.close()
         del blk, tw
     return out
@@ -666,6 +714,58 @@ def run_h3dit(args):
         if ctx.sync_status() != 0:
             raise RuntimeError("end-to-end steps failed")
 
+    # the whole 6-step sampling loop in one call (h3dit_denoise) on the 4096^2
+    # latent [24, 256, 256]: on the device, and end to end with the noise and
+    # the text states copied in from pinned host memory and the denoised
+    # latent copied back, all inside the timed region
+    denoise = None
+    if not args.no_denoise:
+        g = torch.Generator(device="cuda")
+        g.manual_seed(2000 + rank)
+        k4 = 4 * C_LAT
+        rnd = lambda *s: torch.randn(*s, device="cuda", generator=g) * 0.02
+        io = {"w_in": rnd(D, k4), "b_in": torch.zeros(D, device="cuda"), "w_mod": rnd(2 * D, D),
+              "b_mod": torch.zeros(2 * D, device="cuda"), "w_out": rnd(k4, D),
+              "b_out": torch.zeros(k4, device="cuda")}
+        shape = (C_LAT, 2 * GRID, 2 * GRID)
+        noise = torch.randn(*shape, device="cuda", generator=g)
+        lat = torch.empty_like(noise)
+        h_noise = torch.empty(shape, pin_memory=True)
+        h_noise.copy_(noise)
+        h_txt = torch.empty(x_txt.shape, dtype=x_txt.dtype, pin_memory=True)
+        h_txt.copy_(x_txt)
+        h_out = torch.empty(shape, pin_memory=True)
+        lat.copy_(noise)
+        ctx.denoise(io, lat, x_txt, 6)  # warm-up
+        barrier()
+        reps = 2
+        e0.record(stream)
+        for _ in range(reps):
+            lat.copy_(noise)
+            ctx.denoise(io, lat, x_txt, 6)
+        e1.record(stream)
+        barrier()
+        d_ms = slowest_rank(e0.elapsed_time(e1), dist) / reps
+        e0.record(stream)
+        for _ in range(reps):
+            lat.copy_(h_noise, non_blocking=True)
+            x_txt.copy_(h_txt, non_blocking=True)
+            ctx.denoise(io, lat, x_txt, 6)
+            h_out.copy_(lat, non_blocking=True)
+        e1.record(stream)
+        barrier()
+        de_ms = slowest_rank(e0.elapsed_time(e1), dist) / reps
+        if ctx.sync_status() != 0:
+            raise RuntimeError("denoise failed")
+        if not bool(torch.isfinite(h_out).all()):
+            raise RuntimeError("denoise produced non-finite values")
+        in_bytes = h_noise.numel() * 4 + h_txt.numel() * h_txt.element_size()
+        denoise = {"ms": round(d_ms / world, 1), "steps": 6, "latent": list(shape),
+                   "e2e": {"value": round(de_ms / world, 1), "unit": "ms",
+                           "h2d_bytes_per_run": in_bytes,
+                           "d2h_bytes_per_run": h_out.numel() * 4}}
+        del io, noise, lat
+
     line = None
     if rank == 0:
         peaks, peak_src = load_peaks()
@@ -717,6 +817,7 @@ def run_h3dit(args):
             "step_ms": {"median": round(per_step[len(per_step) // 2], 2),
                         "min": round(per_step[0], 2), "max": round(per_step[-1], 2)},
             "six_step_ms": round(6 * ms_step, 1),
+            "denoise_6step": denoise,
             "graph_ms_per_step": None if graph_ms is None else round(graph_ms, 2),
         }
         gemm_kinds = ("qkv", "out_proj", "ffn1", "ffn2")
@@ -725,13 +826,23 @@ def run_h3dit(args):
             g_fl = sum(flops_per_launch(k, N_TOK, dh) * prof[k][1] for k in gemm_kinds)
             line["gemm_tflops"] = round(g_fl / g_ms / 1e9, 1)
             line["attention_tflops"] = kernels.get("attention", {}).get("tflops")
+        line["frac_of_nominal_bf16"] = {
+            "peak_tflops": NOMINAL_BF16_TFLOPS,
+            "step": round(line["tflops_step"] / NOMINAL_BF16_TFLOPS, 4),
+            "gemm": round(line.get("gemm_tflops", 0.0) / NOMINAL_BF16_TFLOPS, 4),
+            "attention": round((line.get("attention_tflops") or 0.0) / NOMINAL_BF16_TFLOPS, 4)}
         if world == 1 and not args.no_configs:
-            line["ms_per_block"] = block_timings(dh)
+            line["ms_per_block"] = block_timings(96)
+            line["ms_per_block"].update(block_timings(128))
         if world == 1 and not args.no_cpu_baseline:
             v, desc, threads, secs = oracle_sample(dh)
             line["cpu_baseline"] = {"value": round(v, 1), "unit": "ms", "cores": threads,
-                                    "kind": "oracle", "sample": desc,
+                                    "kind": "oracle", "estimated": True, "sample": desc,
                                     "sample_cpu_seconds": round(secs, 1)}
+            b_ms, b_desc, b_threads = oracle_block_2k(dh)
+            line["cpu_baseline_block_2k"] = {"value": round(b_ms, 1), "unit": "ms per block",
+                                             "cores": b_threads, "kind": "oracle",
+                                             "estimated": False, "sample": b_desc}
     # the MXFP8 variant (a11), on the same bf16 weights quantized at create
     if not args.no_mxfp8:
         from image_generation_b200 import h3dit as Hb

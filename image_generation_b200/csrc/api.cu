@@ -31,7 +31,7 @@ struct MxWeights {
 constexpr size_t kNoTiled = ~static_cast<size_t>(0);
 
 struct Layout {
-  size_t status, resid, xm, qkv, attn, u, mod, cvec, hidden, rope, wptr, bptr;
+  size_t status, resid, xm, qkv, attn, u, mod, cvec, hidden, omod, rope, wptr, bptr;
   // MXFP8 precision only
   size_t xq, xq_sf, oq, oq_sf, uq, uq_sf, wq, wq_block;
   MxWeights wq_off;  // offsets inside one block's slice of the wq arena
@@ -76,6 +76,7 @@ Layout plan(const h3dit_config *c) {
   L.mod = take(static_cast<size_t>(c->n_blocks) * 6 * D * 4);
   L.cvec = take(D * 4);
   L.hidden = take(D * 4);
+  L.omod = take(2 * D * 4);
   L.rope = take(N * (c->head_dim / 2) * 2 * 4);
   L.wptr = take(static_cast<size_t>(c->n_blocks) * sizeof(void *));
   L.bptr = take(static_cast<size_t>(c->n_blocks) * sizeof(void *));
@@ -164,6 +165,7 @@ struct h3dit_ctx {
   float *mod(int l) { return reinterpret_cast<float *>(ws + L.mod) + static_cast<size_t>(l) * 6 * cfg.hidden; }
   float *cvec() { return reinterpret_cast<float *>(ws + L.cvec); }
   float *hidden() { return reinterpret_cast<float *>(ws + L.hidden); }
+  float *omod() { return reinterpret_cast<float *>(ws + L.omod); }
   float *rope() { return reinterpret_cast<float *>(ws + L.rope); }
   const void *const *wptr() { return reinterpret_cast<const void *const *>(ws + L.wptr); }
   const float *const *bptr() { return reinterpret_cast<const float *const *>(ws + L.bptr); }
@@ -757,6 +759,67 @@ h3dit_status h3dit_rope_table(h3dit_ctx *ctx, const h3dit_grid *grids, int32_t n
                          static_cast<cudaStream_t>(cuda_stream));
 }
 
+namespace {
+// Shape rules shared by the latent entry points: C in [1, 32], even sides,
+// and at most max_tokens tokens.
+h3dit_status check_latent(h3dit_ctx *ctx, const float *latent, int channels, int lat_h,
+                          int lat_w) {
+  if (!latent || !aligned16(latent)) return ctx->fail(H3DIT_ERR_INVALID_ARG, "latent is NULL or misaligned");
+  if (channels < 1 || channels > 32)
+    return ctx->fail(H3DIT_ERR_UNSUPPORTED, "latent channels %d outside [1, 32]", channels);
+  if (lat_h < 2 || lat_w < 2 || (lat_h & 1) || (lat_w & 1))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "latent sides %d x %d must be even and >= 2", lat_h, lat_w);
+  const long long n = static_cast<long long>(lat_h / 2) * (lat_w / 2);
+  if (n > ctx->cfg.max_tokens)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "%lld tokens exceed max_tokens=%d", n, ctx->cfg.max_tokens);
+  return H3DIT_OK;
+}
+}  // namespace
+
+h3dit_status h3dit_embed_latent(h3dit_ctx *ctx, const float *latent, int32_t channels,
+                                int32_t lat_h, int32_t lat_w, const float *w_in, const float *b_in,
+                                void *x_img_out, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  h3dit_status st = check_latent(ctx, latent, channels, lat_h, lat_w);
+  if (st) return st;
+  if (!w_in || !b_in || !x_img_out || !aligned16(w_in) || !aligned16(b_in) || !aligned16(x_img_out))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "embedding: NULL or misaligned pointer");
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  Launch L(ctx, H3DIT_KERNEL_IO, s);
+  return ctx->cuda(launch_embed_latent(latent, channels, lat_h, lat_w, w_in, b_in, ctx->cfg.hidden,
+                                       x_img_out, ctx->cfg.io_fp32 != 0, s),
+                   "embed latent launch");
+}
+
+h3dit_status h3dit_output_modulation(h3dit_ctx *ctx, const float *c, const float *w_mod,
+                                     const float *b_mod, float *mod_out, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (!c || !w_mod || !b_mod || !mod_out)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "output modulation: NULL pointer");
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  Launch L(ctx, H3DIT_KERNEL_IO, s);
+  return ctx->cuda(launch_output_modulation(c, w_mod, b_mod, mod_out, ctx->cfg.hidden, s),
+                   "output modulation launch");
+}
+
+h3dit_status h3dit_output_euler(h3dit_ctx *ctx, const void *x_img, const float *mod,
+                                const float *w_out, const float *b_out, float *latent,
+                                int32_t channels, int32_t lat_h, int32_t lat_w, float dt,
+                                void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  h3dit_status st = check_latent(ctx, latent, channels, lat_h, lat_w);
+  if (st) return st;
+  if (!x_img || !mod || !w_out || !b_out)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "output layer: NULL pointer");
+  if (!(dt == dt)) return ctx->fail(H3DIT_ERR_INVALID_ARG, "dt is NaN");
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  Launch L(ctx, H3DIT_KERNEL_IO, s, 2);
+  return ctx->cuda(launch_output_euler(x_img, ctx->cfg.io_fp32 != 0, mod, w_out, b_out,
+                                       ctx->cfg.hidden, ctx->cfg.norm_eps, latent, channels, lat_h,
+                                       lat_w, dt, ctx->resid(), s),
+                   "output layer launch");
+}
+
 h3dit_status h3dit_linear(h3dit_ctx *ctx, int32_t epilogue, const void *a, const void *w,
                           int32_t m, int32_t n, int32_t k, void *out, const float *gate,
                           const float *rope_table, void *cuda_stream) {
@@ -812,6 +875,66 @@ h3dit_status h3dit_step(h3dit_ctx *ctx, float t, void *x_img, const h3dit_grid *
   return run_unpack(ctx, n_txt, n_img, x_txt, x_img, s);
 }
 
+h3dit_status h3dit_denoise(h3dit_ctx *ctx, const h3dit_io_weights *io, float *latent,
+                           int32_t channels, int32_t lat_h, int32_t lat_w, const void *x_txt,
+                           int32_t n_txt, int32_t n_steps, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (!io || !io->w_in || !io->b_in || !io->w_mod || !io->b_mod || !io->w_out || !io->b_out ||
+      !aligned16(io->w_in) || !aligned16(io->b_in))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "denoise: NULL or misaligned FP32 layer weights");
+  h3dit_status st = check_latent(ctx, latent, channels, lat_h, lat_w);
+  if (st) return st;
+  if (n_steps < 1 || n_steps > 1000)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "n_steps %d outside [1, 1000]", n_steps);
+  if (n_txt < 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "n_txt < 0");
+  if (n_txt > 0 && (!x_txt || !aligned16(x_txt)))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "x_txt is NULL or misaligned");
+  const int D = ctx->cfg.hidden;
+  const int h = lat_h / 2, w = lat_w / 2;
+  const long long n = static_cast<long long>(n_txt) + static_cast<long long>(h) * w;
+  if (n > ctx->cfg.max_tokens)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "%lld tokens exceed max_tokens=%d", n, ctx->cfg.max_tokens);
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  const h3dit_grid grid{0, h, w};
+  if ((st = rope_table_into(ctx, &grid, 1, n_txt, static_cast<int>(n), ctx->rope(), s))) return st;
+  // the image rows of the packed fp32 residual stream [text; image]
+  float *x_img = ctx->resid() + static_cast<size_t>(n_txt) * D;
+  // the FFN hidden buffer is free once the blocks have run: one float per
+  // image token of it holds the output layer's row scales
+  float *rinv = static_cast<float *>(ctx->u());
+  for (int k = 0; k < n_steps; ++k) {
+    const double tk = 1.0 - static_cast<double>(k) / n_steps;
+    const double tn = 1.0 - static_cast<double>(k + 1) / n_steps;
+    const float t = static_cast<float>(tk);
+    if ((st = h3dit_time_embed(ctx, t, ctx->cvec(), s))) return st;
+    if ((st = h3dit_adaln_project(ctx, ctx->cvec(), 0, ctx->cfg.n_blocks, ctx->mod(0), s))) return st;
+    {
+      Launch L(ctx, H3DIT_KERNEL_IO, s);
+      if ((st = ctx->cuda(launch_output_modulation(ctx->cvec(), io->w_mod, io->b_mod, ctx->omod(),
+                                                   D, s),
+                          "output modulation launch")))
+        return st;
+    }
+    if (n_txt > 0 && (st = run_pack(ctx, x_txt, n_txt, nullptr, 0, s))) return st;
+    {
+      Launch L(ctx, H3DIT_KERNEL_IO, s);
+      if ((st = ctx->cuda(launch_embed_latent(latent, channels, lat_h, lat_w, io->w_in, io->b_in,
+                                              D, x_img, true, s),
+                          "embed latent launch")))
+        return st;
+    }
+    for (int l = 0; l < ctx->cfg.n_blocks; ++l)
+      if ((st = block_body(ctx, l, ctx->mod(l), static_cast<int>(n), s))) return st;
+    Launch L(ctx, H3DIT_KERNEL_IO, s, 2);
+    if ((st = ctx->cuda(launch_output_euler(x_img, true, ctx->omod(), io->w_out, io->b_out, D,
+                                            ctx->cfg.norm_eps, latent, channels, lat_h, lat_w,
+                                            static_cast<float>(tn - tk), rinv, s),
+                        "output layer launch")))
+      return st;
+  }
+  return H3DIT_OK;
+}
+
 size_t h3dit_mx_scale_bytes(int32_t rows, int32_t k) {
   if (rows <= 0 || k <= 0 || k % 128) return 0;
   return mx_sf_bytes(rows, k);
@@ -824,7 +947,7 @@ h3dit_status h3dit_mx_quantize(h3dit_ctx *ctx, const void *src, int32_t rows, in
     return ctx->fail(H3DIT_ERR_UNSUPPORTED, "MXFP8 quantization needs k a multiple of 128");
   if (!src || !dst || !sf || !aligned16(src) || !aligned16(dst))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "NULL or misaligned pointer");
-  Launch L(ctx, H3DIT_KERNEL_PACK, static_cast<cudaStream_t>(cuda_stream));
+  Launch L(ctx, H3DIT_KERNEL_MX_QUANTIZE, static_cast<cudaStream_t>(cuda_stream));
   return ctx->cuda(launch_mx_quantize(src, k, rows, k, static_cast<uint8_t *>(dst),
                                       static_cast<uint8_t *>(sf),
                                       static_cast<cudaStream_t>(cuda_stream)),

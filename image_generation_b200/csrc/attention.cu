@@ -375,13 +375,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 template <int DH, bool OUT_MX>
 cudaError_t launch_dh(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
                       const AttnParams &p, int heads, cudaStream_t s) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tcgen05<DH, OUT_MX>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static PerDevice smem_attr;
+  cudaError_t e = set_smem_once(smem_attr, attn_fwd_tcgen05<DH, OUT_MX>, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
   dim3 grid((p.n + 2 * BQ - 1) / (2 * BQ), heads);
   attn_fwd_tcgen05<DH, OUT_MX><<<grid, THREADS, SMEM_BYTES, s>>>(q, k, v, p);
   return cudaGetLastError();

@@ -191,13 +191,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 template <int EPI>
 cudaError_t launch_one(const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p, int grid,
                        cudaStream_t s) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05<EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static PerDevice smem_attr;
+  cudaError_t e = set_smem_once(smem_attr, gemm_bf16_tcgen05<EPI>, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
   gemm_bf16_tcgen05<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(a, b, p);
   return cudaGetLastError();
 }

@@ -238,13 +238,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 template <int EPI>
 cudaError_t launch_one(const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p, int grid,
                        cudaStream_t s) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_pair<EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static PerDevice smem_attr;
+  cudaError_t e = set_smem_once(smem_attr, gemm_bf16_pair<EPI>, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(THREADS, 1, 1);
@@ -261,12 +257,30 @@ cudaError_t launch_one(const CUtensorMap &a, const CUtensorMap &b, const GemmPar
 }
 
 template <int EPI>
+int occupancy_clusters();
+
+// Clusters that fit at once on the current device, found once per device (0
+// when the kernel cannot be configured there).
+template <int EPI>
 int max_pairs_for() {
-  static int cached = -1;
-  if (cached >= 0) return cached;
-  if (cudaFuncSetAttribute(gemm_bf16_pair<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           SMEM_BYTES) != cudaSuccess)
-    return cached = 0;
+  static PerDevice pairs;
+  int n = 0;
+  if (per_device(pairs, [](int *v) {
+        *v = 0;
+        if (cudaFuncSetAttribute(gemm_bf16_pair<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SMEM_BYTES) != cudaSuccess) {
+          cudaGetLastError();
+          return cudaSuccess;
+        }
+        *v = occupancy_clusters<EPI>();
+        return cudaSuccess;
+      }, &n) != cudaSuccess)
+    return 0;
+  return n;
+}
+
+template <int EPI>
+int occupancy_clusters() {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(2, 1, 1);
   cfg.blockDim = dim3(THREADS, 1, 1);
@@ -279,8 +293,11 @@ int max_pairs_for() {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_bf16_pair<EPI>, &cfg) != cudaSuccess) n = 0;
-  return cached = n;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_bf16_pair<EPI>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  return n;
 }
 
 }  // namespace

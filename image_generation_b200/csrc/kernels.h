@@ -5,7 +5,56 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 namespace h3 {
+
+// A value computed once per device for the whole process (a kernel attribute
+// such as the dynamic shared-memory limit takes effect only on the device
+// that is current when it is set, and occupancy differs between devices).
+// Each launcher keeps one of these per kernel instance; the first launch on a
+// device computes it under a lock, later ones read it without one, so host
+// threads that drive different devices may race on first use.
+constexpr int kMaxDevices = 64;
+struct PerDevice {
+  std::mutex mu;
+  std::atomic<int> value[kMaxDevices];
+  PerDevice() {
+    for (auto &v : value) v.store(-1, std::memory_order_relaxed);
+  }
+};
+// Runs `compute(int *v)` on the current device unless it has succeeded there
+// before; *out (optional) receives the stored value (>= 0).
+template <typename F>
+inline cudaError_t per_device(PerDevice &pd, F &&compute, int *out = nullptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  int v = pd.value[dev].load(std::memory_order_acquire);
+  if (v < 0) {
+    std::lock_guard<std::mutex> lock(pd.mu);
+    v = pd.value[dev].load(std::memory_order_relaxed);
+    if (v < 0) {
+      int got = 0;
+      e = compute(&got);
+      if (e != cudaSuccess) return e;
+      v = got < 0 ? 0 : got;
+      pd.value[dev].store(v, std::memory_order_release);
+    }
+  }
+  if (out) *out = v;
+  return cudaSuccess;
+}
+// The common case: raise a kernel's dynamic shared-memory limit once per device.
+template <typename K>
+inline cudaError_t set_smem_once(PerDevice &pd, K *kernel, int bytes) {
+  return per_device(pd, [&](int *v) {
+    *v = 1;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  });
+}
 
 enum Epilogue : int {
   kEpiStore = 0,
@@ -96,6 +145,16 @@ inline size_t mx_sf_tiled_bytes(long long n, long long k) {
 }
 cudaError_t launch_gemm_mx(const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p,
                            int epilogue, int grid, bool wide, cudaStream_t s);
+// Around the block loop (io_layers.cu): 2x2 patchify + FP32 embedding into
+// tokens; the output layer's modulation; output layer + unpatchify + Euler.
+cudaError_t launch_embed_latent(const float *z, int C, int Hl, int Wl, const float *w_in,
+                                const float *b_in, int D, void *out, bool out_fp32,
+                                cudaStream_t s);
+cudaError_t launch_output_modulation(const float *c, const float *w_mod, const float *b_mod,
+                                     float *mod, int D, cudaStream_t s);
+cudaError_t launch_output_euler(const void *x, bool in_fp32, const float *mod, const float *w_out,
+                                const float *b_out, int D, float eps, float *z, int C, int Hl,
+                                int Wl, float dt, float *rinv_scratch, cudaStream_t s);
 cudaError_t launch_mx_tile_sf(const uint8_t *sf, int n, int k, uint8_t *tiled, cudaStream_t s);
 // bf16 [rows, k] (row stride ld elements) -> E4M3 [rows, k] + scales.
 cudaError_t launch_mx_quantize(const void *src, long long ld, int rows, int k, uint8_t *dst,

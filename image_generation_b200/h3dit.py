@@ -38,7 +38,7 @@ H3DIT_PRECISION_MXFP8 = 1
 H3DIT_STATIC_TIME_MAX_HIDDEN = 8192
 
 KERNEL_KINDS = ["time_embed", "adaln", "rmsnorm", "qkv", "attention", "out_proj", "ffn1",
-                "ffn2", "rope_table", "pack"]
+                "ffn2", "rope_table", "pack", "mx_quantize", "io"]
 
 
 class h3dit_config(C.Structure):
@@ -59,6 +59,11 @@ class h3dit_time_weights(C.Structure):
 class h3dit_block_weights(C.Structure):
     _fields_ = [("w_qkv", C.c_void_p), ("w_o", C.c_void_p), ("w_ff1", C.c_void_p),
                 ("w_ff2", C.c_void_p), ("w_ada", C.c_void_p), ("b_ada", C.c_void_p)]
+
+
+class h3dit_io_weights(C.Structure):
+    _fields_ = [("w_in", C.c_void_p), ("b_in", C.c_void_p), ("w_mod", C.c_void_p),
+                ("b_mod", C.c_void_p), ("w_out", C.c_void_p), ("b_out", C.c_void_p)]
 
 
 class h3dit_grid(C.Structure):
@@ -100,6 +105,11 @@ def _load() -> C.CDLL:
         "h3dit_block_linear_mx": (i32, [p, i32, i32, p, p, i32, p, p, p, p, p]),
         "h3dit_rmsnorm_modulate_mx": (i32, [p, p, p, p, p, p, i32, p]),
         "h3dit_attention_mx": (i32, [p, p, p, p, i32, p, p, i32, p]),
+        "h3dit_embed_latent": (i32, [p, p, i32, i32, i32, p, p, p, p]),
+        "h3dit_output_modulation": (i32, [p, p, p, p, p, p]),
+        "h3dit_output_euler": (i32, [p, p, p, p, p, p, i32, i32, i32, f32, p]),
+        "h3dit_denoise": (i32, [p, C.POINTER(h3dit_io_weights), p, i32, i32, i32, p, i32, i32,
+                                p]),
         "h3dit_selftest_bounded_wait": (i32, [p, i32, p]),
         "h3dit_profile_begin": (i32, [p]),
         "h3dit_profile_end": (i32, [p, C.POINTER(C.c_float), C.POINTER(C.c_int64)]),
@@ -190,7 +200,11 @@ def _stream(stream=None) -> int:
 class Context:
     """Owns one h3dit_ctx plus the torch tensors it borrows (weights, workspace)."""
 
-    def __init__(self, cfg: h3dit_config, time_w: dict, blocks: Sequence[dict], stream=None):
+    def __init__(self, cfg: h3dit_config, time_w: dict, blocks: Sequence[dict], stream=None,
+                 workspace=None):
+        """workspace: optional caller-owned uint8 device tensor of at least
+        h3dit_workspace_bytes(cfg) bytes (256-byte aligned); allocated here
+        when omitted."""
         import torch
 
         self.cfg = cfg
@@ -198,7 +212,11 @@ class Context:
         ws_bytes = lib.h3dit_workspace_bytes(C.byref(cfg))
         if ws_bytes == 0:
             raise H3DitError(H3DIT_ERR_INVALID_ARG, "invalid config")
-        self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        if workspace is None:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        elif workspace.numel() * workspace.element_size() < ws_bytes:
+            raise H3DitError(H3DIT_ERR_WORKSPACE, "workspace smaller than h3dit_workspace_bytes")
+        self.workspace = workspace
         tw = h3dit_time_weights(_ptr(time_w["w_t1"]), _ptr(time_w["b_t1"]),
                                 _ptr(time_w["w_t2"]), _ptr(time_w["b_t2"]))
         arr = (h3dit_block_weights * len(blocks))()
@@ -206,7 +224,7 @@ class Context:
             arr[i] = h3dit_block_weights(_ptr(b["w_qkv"]), _ptr(b["w_o"]), _ptr(b["w_ff1"]),
                                          _ptr(b["w_ff2"]), _ptr(b["w_ada"]), _ptr(b["b_ada"]))
         handle = C.c_void_p()
-        st = lib.h3dit_create(C.byref(cfg), C.byref(tw), arr, self.workspace.data_ptr(),
+        st = lib.h3dit_create(C.byref(cfg), C.byref(tw), arr, _ptr(self.workspace),
                               ws_bytes, _stream(stream), C.byref(handle))
         check(None, st)
         self.handle = handle
@@ -287,6 +305,33 @@ class Context:
         self._check(lib.h3dit_attention_mx(self.handle, _ptr(q, False), _ptr(k, False),
                                            _ptr(v, False), ld_qkv, _ptr(o), _ptr(o_sf), n,
                                            _stream(stream)))
+
+    def embed_latent(self, latent, w_in, b_in, x_img_out, stream=None) -> None:
+        """latent fp32 [C, Hl, Wl] -> x_img_out [(Hl/2)(Wl/2), D] in the token dtype."""
+        ch, h, w = latent.shape
+        self._check(lib.h3dit_embed_latent(self.handle, _ptr(latent), ch, h, w, _ptr(w_in),
+                                           _ptr(b_in), _ptr(x_img_out), _stream(stream)))
+
+    def output_modulation(self, c, w_mod, b_mod, mod_out, stream=None) -> None:
+        self._check(lib.h3dit_output_modulation(self.handle, _ptr(c), _ptr(w_mod), _ptr(b_mod),
+                                                _ptr(mod_out), _stream(stream)))
+
+    def output_euler(self, x_img, mod, w_out, b_out, latent, dt: float, stream=None) -> None:
+        """latent += dt * unpatchify(output layer(x_img)), in place."""
+        ch, h, w = latent.shape
+        self._check(lib.h3dit_output_euler(self.handle, _ptr(x_img), _ptr(mod), _ptr(w_out),
+                                           _ptr(b_out), _ptr(latent), ch, h, w, dt,
+                                           _stream(stream)))
+
+    def denoise(self, io: dict, latent, x_txt, n_steps: int, stream=None) -> None:
+        """latent fp32 [C, Hl, Wl]: noise in, the latent after n_steps Euler
+        steps out; io holds w_in, b_in, w_mod, b_mod, w_out, b_out."""
+        ch, h, w = latent.shape
+        iw = h3dit_io_weights(_ptr(io["w_in"]), _ptr(io["b_in"]), _ptr(io["w_mod"]),
+                              _ptr(io["b_mod"]), _ptr(io["w_out"]), _ptr(io["b_out"]))
+        n_txt = 0 if x_txt is None else x_txt.shape[0]
+        self._check(lib.h3dit_denoise(self.handle, C.byref(iw), _ptr(latent), ch, h, w,
+                                      _ptr(x_txt), n_txt, n_steps, _stream(stream)))
 
     def selftest_bounded_wait(self, limit_us: int, stream=None) -> None:
         self._check(lib.h3dit_selftest_bounded_wait(self.handle, limit_us, _stream(stream)))

@@ -255,6 +255,75 @@ h3dit_status h3dit_rmsnorm_modulate_mx(h3dit_ctx *ctx, const float *x, const flo
 h3dit_status h3dit_attention_mx(h3dit_ctx *ctx, const void *q, const void *k, const void *v,
                                 int32_t ld_qkv, void *o, void *o_sf, int32_t n, void *cuda_stream);
 
+/* ---- Around the block loop: latent in, velocity out, sampler step --------
+ * MiniMax-H3-Image model card, "Model Architecture": the image VAE's latent
+ * has 24 channels at 16x spatial downsampling; the DiT patchifies it with a
+ * 2x2 patch (one token per 32x32 pixels); the embedding, timestep and output
+ * layers are FP32. The real per-step output heads and sampling schedule are
+ * not on the pages; a DiT output layer predicting the flow velocity dz/dt and
+ * an Euler step stand in for them.
+ * Latents are device fp32 [C, Hl, Wl] (channel-major), Hl and Wl even, C <= 32.
+ * Token (r, c) of a latent is row-major over its (Hl/2, Wl/2) patch grid, the
+ * order h3dit_grid gives an image; feature ch*4 + 2i + j of a token is latent
+ * pixel (2r + i, 2c + j) of channel ch. */
+
+/* Patchify + FP32 patch embedding: x_img_out[t] = W_in patch(t) + b_in.
+ *   w_in device fp32 [D, 4C]; b_in device fp32 [D];
+ *   x_img_out device [(Hl/2)(Wl/2), D] in the context's token dtype (bf16,
+ *   or fp32 with io_fp32), ready for h3dit_step as the target image. */
+h3dit_status h3dit_embed_latent(h3dit_ctx *ctx, const float *latent, int32_t channels,
+                                int32_t lat_h, int32_t lat_w, const float *w_in, const float *b_in,
+                                void *x_img_out, void *cuda_stream);
+
+/* The output layer's modulation: mod_out[0:D] = shift, mod_out[D:2D] = scale,
+ * = W_mod SiLU(c) + b_mod. c device fp32 [D] (h3dit_time_embed's output);
+ * w_mod device fp32 [2D, D]; b_mod [2D]; mod_out device fp32 [2D]. */
+h3dit_status h3dit_output_modulation(h3dit_ctx *ctx, const float *c, const float *w_mod,
+                                     const float *b_mod, float *mod_out, void *cuda_stream);
+
+/* Output layer, unpatchify and one Euler step of the flow, in place on the
+ * latent: v = unpatchify((RMSNorm(x) (1 + scale) + shift) W_out^T + b_out);
+ * latent += dt * v (dt = t_next - t, negative when denoising from t = 1 to 0).
+ *   x_img device [(Hl/2)(Wl/2), D], the target image's tokens after h3dit_step,
+ *   in the context's token dtype; mod device fp32 [2D] from
+ *   h3dit_output_modulation; w_out device fp32 [4C, D]; b_out [4C].
+ * Uses the context's residual workspace as scratch (one float per token). */
+h3dit_status h3dit_output_euler(h3dit_ctx *ctx, const void *x_img, const float *mod,
+                                const float *w_out, const float *b_out, float *latent,
+                                int32_t channels, int32_t lat_h, int32_t lat_w, float dt,
+                                void *cuda_stream);
+
+/* The FP32 layers around the block loop, for h3dit_denoise (C = latent
+ * channels; all device fp32, nn.Linear layout). */
+typedef struct h3dit_io_weights {
+  const float *w_in;  /* [D, 4C] patch embedding      */
+  const float *b_in;  /* [D]                          */
+  const float *w_mod; /* [2D, D] output modulation    */
+  const float *b_mod; /* [2D]  (shift rows, then scale rows) */
+  const float *w_out; /* [4C, D] output layer         */
+  const float *b_out; /* [4C]                         */
+} h3dit_io_weights;
+
+/* The whole sampling loop on one target latent, in place: n_steps Euler steps
+ * of the flow from t = 1 (noise) to t = 0 at t_k = 1 - k / n_steps (the model
+ * card's "6 sampling steps" with the plain uniform schedule; the real schedule
+ * file is not on the pages). Each step runs, all on `cuda_stream`:
+ *   the timestep MLP and every block's AdaLN projection at t_k, and the output
+ *   layer's modulation; the text states x_txt and the patch embedding of the
+ *   latent packed into the fp32 residual stream [text; image]; the n_blocks
+ *   blocks; the output layer on the image rows; latent += (t_{k+1} - t_k) v.
+ *   latent  device fp32 [C, Hl, Wl], noise in, denoised latent out; Hl, Wl
+ *           even, C <= 32; the target image is frame 0 of grid (Hl/2, Wl/2);
+ *   x_txt   device [n_txt, D] in the context's token dtype, read only (the
+ *           same text states enter every step); NULL when n_txt == 0;
+ *   n_steps 1 .. 1000.
+ * Needs n_txt + (Hl/2)(Wl/2) <= max_tokens. The token buffers of h3dit_step
+ * are not used: the residual stream stays in the workspace between the
+ * embedding and the output layer. */
+h3dit_status h3dit_denoise(h3dit_ctx *ctx, const h3dit_io_weights *io, float *latent,
+                           int32_t channels, int32_t lat_h, int32_t lat_w, const void *x_txt,
+                           int32_t n_txt, int32_t n_steps, void *cuda_stream);
+
 /* ---- Timestep condition without any device allocation ----------------- */
 
 /* Largest `hidden` h3dit_time_embed_static accepts. */
@@ -310,7 +379,9 @@ h3dit_status h3dit_selftest_bounded_wait(h3dit_ctx *ctx, int32_t limit_us, void 
 #define H3DIT_KERNEL_FFN2 7       /* a9                            */
 #define H3DIT_KERNEL_ROPE_TABLE 8 /* RoPE table of the sequence    */
 #define H3DIT_KERNEL_PACK 9       /* packing / unpacking tokens    */
-#define H3DIT_KERNEL_COUNT 10
+#define H3DIT_KERNEL_MX_QUANTIZE 10 /* h3dit_mx_quantize           */
+#define H3DIT_KERNEL_IO 11        /* patch embedding, output layer + Euler */
+#define H3DIT_KERNEL_COUNT 12
 
 /* Start recording a CUDA event pair around every kernel the context launches
  * (on the stream it is launched on), dropping earlier records. */

@@ -21,6 +21,21 @@ def test_library_exports_every_declared_function():
         assert hasattr(H.lib, f)
 
 
+def test_profile_kinds_match_the_header():
+    """The binding names one profile slot per H3DIT_KERNEL_* value, in order."""
+    import re
+
+    with open(H.HEADER) as fh:
+        text = fh.read()
+    kinds = {m.group(1): int(m.group(2))
+             for m in re.finditer(r"#define H3DIT_KERNEL_([A-Z_0-9]+)\s+(\d+)", text)}
+    count = kinds.pop("COUNT")
+    assert count == len(H.KERNEL_KINDS)
+    assert sorted(kinds.values()) == list(range(count))
+    by_value = {v: k.lower() for k, v in kinds.items()}
+    assert [by_value[i] for i in range(count)] == H.KERNEL_KINDS
+
+
 def test_status_strings():
     for s in (H.H3DIT_OK, H.H3DIT_ERR_INVALID_ARG, H.H3DIT_ERR_UNSUPPORTED,
               H.H3DIT_ERR_WORKSPACE, H.H3DIT_ERR_CUDA, H.H3DIT_ERR_TIMEOUT):
@@ -115,6 +130,15 @@ def test_null_context_is_rejected_everywhere():
         == H.H3DIT_ERR_INVALID_ARG
     assert H.lib.h3dit_block_linear_mx(None, 0, H.H3DIT_LINEAR_QKV, 0x10000, 0x10000, 4, 0x10000,
                                        None, None, 0x10000, None) == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_embed_latent(None, 0x10000, 24, 4, 4, 0x10000, 0x10000, 0x10000, None) \
+        == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_output_modulation(None, 0x10000, 0x10000, 0x10000, 0x10000, None) \
+        == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_output_euler(None, 0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 24, 4, 4,
+                                    -0.1, None) == H.H3DIT_ERR_INVALID_ARG
+    io = H.h3dit_io_weights(0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 0x10000)
+    assert H.lib.h3dit_denoise(None, C.byref(io), 0x10000, 24, 4, 4, 0x10000, 8, 6, None) \
+        == H.H3DIT_ERR_INVALID_ARG
     H.lib.h3dit_destroy(None)  # NULL-safe
     assert H.lib.h3dit_last_error(None) == b"no context"
 

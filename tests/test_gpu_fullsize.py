@@ -27,7 +27,8 @@ def _check_rows(y, x, ref, rows, what):
     assert_delta_close(y[rows] - x[rows], ref - x[rows], what + " (branch delta)")
 
 
-@pytest.mark.parametrize("name", ["block_2k", "block_2k_dh128", "block_4k", "edit_4ref"])
+@pytest.mark.parametrize("name", ["block_2k", "block_2k_dh128", "block_4k", "block_4k_dh128",
+                                  "edit_4ref", "edit_4ref_dh128"])
 def test_full_width_block_sampled_rows(name):
     from image_generation_b200 import h3dit as H
 
