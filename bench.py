@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-mxfp8", action="store_true")
+    ap.add_argument("--no-streaming", action="store_true",
+                    help="skip the layerwise weight-streaming timings")
     ap.add_argument("--no-denoise", action="store_true",
                     help="skip the 6-step sampling loop timing (h3dit_denoise)")
     ap.add_argument("--no-graph", action="store_true", help="skip the graph-replayed step timing")
@@ -603,6 +605,49 @@ def block_timings(dh: int) -> dict:
     return out
 
 
+def streaming_timings(tw, blocks, x_txt, x_img, grids, dh, residents=(24, 8), steps=2,
+                      host_copies=4):
+    """The 50-block 4096^2 step with only the first k blocks' weights on the
+    device and the rest streamed from pinned host memory through two staging
+    slots (h3dit_attach_staging). The host blocks cycle through
+    `host_copies` distinct pinned copies of the model's own blocks (the bytes
+    moved per step are the same as with 50 - k distinct blocks; the step's
+    output is not compared here - the tests check streamed steps bit for bit
+    against resident ones). Returns {k: ms per step, ...} with the bytes
+    crossing PCIe per step."""
+    import torch
+
+    from image_generation_b200 import h3dit as Hb
+
+    host = [{k: v.cpu().pin_memory() for k, v in blocks[L - 1 - i].items()}
+            for i in range(host_copies)]
+    block_bytes = sum(v.numel() * v.element_size() for v in host[0].values())
+    out = {}
+    for k in residents:
+        mixed = [blocks[l] if l < k else host[l % host_copies] for l in range(L)]
+        ctx = Hb.Context(Hb.make_config(D, H, dh, F, L, N_TOK), tw, mixed)
+        ctx.attach_staging()
+        ts = timesteps(steps + 1)
+        ctx.step(ts[0], x_img, grids, x_txt)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(steps):
+            ctx.step(ts[i + 1], x_img, grids, x_txt)
+        e1.record()
+        torch.cuda.synchronize()
+        if ctx.sync_status() != 0:
+            raise RuntimeError(f"streamed step failed (k={k})")
+        ms = e0.elapsed_time(e1) / steps
+        moved = (L - k) * block_bytes
+        out[f"resident_{k}"] = {"ms_per_step": round(ms, 1), "streamed_blocks": L - k,
+                                "h2d_bytes_per_step": moved,
+                                "h2d_gbs": round(moved / ms / 1e6, 1)}
+        ctx.close()
+    del host
+    return out
+
+
 def block_flops(n: int, d) -> float:
     I = d.heads * d.head_dim
     return 8.0 * n * d.hidden * I + 4.0 * n * d.hidden * d.ffn + 4.0 * n * n * I
@@ -766,6 +811,12 @@ def run_h3dit(args):
                            "d2h_bytes_per_run": h_out.numel() * 4}}
         del io, noise, lat
 
+    streaming = None
+    if world == 1 and not args.no_streaming:
+        streaming = streaming_timings(tw, blocks, x_txt, x_img, grids, dh)
+        streaming["resident_50"] = {"ms_per_step": round(ms_step, 1), "streamed_blocks": 0,
+                                    "h2d_bytes_per_step": 0}
+
     line = None
     if rank == 0:
         peaks, peak_src = load_peaks()
@@ -818,6 +869,7 @@ def run_h3dit(args):
                         "min": round(per_step[0], 2), "max": round(per_step[-1], 2)},
             "six_step_ms": round(6 * ms_step, 1),
             "denoise_6step": denoise,
+            "weight_streaming": streaming,
             "graph_ms_per_step": None if graph_ms is None else round(graph_ms, 2),
         }
         gemm_kinds = ("qkv", "out_proj", "ffn1", "ffn2")

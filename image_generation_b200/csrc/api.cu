@@ -115,6 +115,33 @@ Layout plan(const h3dit_config *c) {
   return L;
 }
 
+// Layerwise weight streaming: two slots, each holding one block's weights
+// (same layout as h3dit_block_weights), then a table of the two slots' w_ada
+// and b_ada pointers for the AdaLN kernel.
+struct Staging {
+  size_t part[6];  // offsets in a slot: w_qkv, w_o, w_ff1, w_ff2, w_ada, b_ada
+  size_t bytes[6]; // bytes of each part
+  size_t slot;     // bytes of one slot
+  size_t table;    // offset of the pointer table (2 x w_ada, then 2 x b_ada)
+  size_t total;
+};
+
+Staging staging_plan(const h3dit_config *c) {
+  Staging S{};
+  const size_t D = c->hidden, I = static_cast<size_t>(c->heads) * c->head_dim, F = c->ffn;
+  const size_t b[6] = {3 * I * D * 2, D * I * 2, F * D * 2, D * F * 2, 6 * D * D * 2, 6 * D * 4};
+  size_t off = 0;
+  for (int i = 0; i < 6; ++i) {
+    S.part[i] = off;
+    S.bytes[i] = b[i];
+    off = round_up(off + b[i], kAlign);
+  }
+  S.slot = off;
+  S.table = 2 * S.slot;
+  S.total = S.table + kAlign;
+  return S;
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -155,6 +182,15 @@ struct h3dit_ctx {
   Layout L{};
   int num_sms = 148;
   std::string err;
+  // layerwise weight streaming: blocks whose weights are pinned host memory
+  std::vector<uint8_t> streamed;  // per block: 1 = weights in host memory
+  int n_streamed = 0;
+  uint8_t *staging = nullptr;     // two slots + pointer table (h3dit_attach_staging)
+  Staging SP{};
+  cudaStream_t copy = nullptr;
+  bool own_copy = false;
+  cudaEvent_t fork = nullptr, join = nullptr, ready[2] = {nullptr, nullptr},
+              slot_free[2] = {nullptr, nullptr};
 
   int *status() { return reinterpret_cast<int *>(ws + L.status); }
   float *resid() { return reinterpret_cast<float *>(ws + L.resid); }
@@ -203,9 +239,26 @@ struct h3dit_ctx {
     }
     records.clear();
   }
+  h3dit_block_weights slot_weights(int s) const {
+    uint8_t *b = staging + static_cast<size_t>(s) * SP.slot;
+    return {b + SP.part[0], b + SP.part[1], b + SP.part[2], b + SP.part[3], b + SP.part[4],
+            reinterpret_cast<const float *>(b + SP.part[5])};
+  }
+  void release_streaming() {
+    for (cudaEvent_t *e : {&fork, &join, &ready[0], &ready[1], &slot_free[0], &slot_free[1]})
+      if (*e) {
+        cudaEventDestroy(*e);
+        *e = nullptr;
+      }
+    if (own_copy && copy) cudaStreamDestroy(copy);
+    copy = nullptr;
+    own_copy = false;
+    staging = nullptr;
+  }
   ~h3dit_ctx() {
     recycle_records();
     for (cudaEvent_t e : event_pool) cudaEventDestroy(e);
+    release_streaming();
   }
 };
 
@@ -431,19 +484,23 @@ h3dit_status run_linear_mx(h3dit_ctx *ctx, int epi, const void *a, const void *a
 }
 
 h3dit_status run_attention(h3dit_ctx *ctx, const void *q, const void *k, const void *v, int ld,
-                           void *o, int ldo, int n, cudaStream_t s, void *o_sf = nullptr) {
+                           void *o, int ldo, int n, cudaStream_t s, void *o_sf = nullptr,
+                           int heads = 0) {
+  if (heads == 0) heads = ctx->cfg.heads;
   if (n < 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "n < 0");
+  if (heads < 1 || heads > ctx->cfg.heads)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "heads %d outside [1, %d]", heads, ctx->cfg.heads);
   if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "attention: NULL or misaligned pointer");
-  const int I = ctx->inner();
+  const int I = heads * ctx->cfg.head_dim;
   if (ld < I || ld % 8 || ldo < I || ldo % 8)
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "attention: row strides must be >= heads*head_dim and multiples of 8");
   if (n == 0) return H3DIT_OK;
   CUtensorMap tq, tk, tv;
   h3dit_status st;
-  if ((st = encode_heads(ctx, &tq, q, n, ctx->cfg.heads, ctx->cfg.head_dim, ld, kAttnBQ))) return st;
-  if ((st = encode_heads(ctx, &tk, k, n, ctx->cfg.heads, ctx->cfg.head_dim, ld, kAttnBKV))) return st;
-  if ((st = encode_heads(ctx, &tv, v, n, ctx->cfg.heads, ctx->cfg.head_dim, ld, kAttnBKV))) return st;
+  if ((st = encode_heads(ctx, &tq, q, n, heads, ctx->cfg.head_dim, ld, kAttnBQ))) return st;
+  if ((st = encode_heads(ctx, &tk, k, n, heads, ctx->cfg.head_dim, ld, kAttnBKV))) return st;
+  if ((st = encode_heads(ctx, &tv, v, n, heads, ctx->cfg.head_dim, ld, kAttnBKV))) return st;
   AttnParams p{};
   p.n = n;
   p.tiles_kv = (n + kAttnBKV - 1) / kAttnBKV;
@@ -455,7 +512,7 @@ h3dit_status run_attention(h3dit_ctx *ctx, const void *q, const void *k, const v
   if (o_sf && (ldo != I || I % 128 || !aligned16(o_sf)))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "MXFP8 attention output needs ld_o == heads*head_dim, a multiple of 128");
   Launch L(ctx, H3DIT_KERNEL_ATTENTION, s);
-  return ctx->cuda(launch_attention(tq, tk, tv, p, ctx->cfg.head_dim, ctx->cfg.heads, o_sf != nullptr, s),
+  return ctx->cuda(launch_attention(tq, tk, tv, p, ctx->cfg.head_dim, heads, o_sf != nullptr, s),
                    "attention launch");
 }
 
@@ -545,9 +602,9 @@ h3dit_status block_body_mx(h3dit_ctx *ctx, int l, const float *mod, int n, cudaS
 }
 
 // Steps a3..a9 on the packed fp32 residual of n tokens (workspace).
-h3dit_status block_body(h3dit_ctx *ctx, int l, const float *mod, int n, cudaStream_t s) {
+h3dit_status block_body(h3dit_ctx *ctx, int l, const h3dit_block_weights &w, const float *mod,
+                        int n, cudaStream_t s) {
   if (ctx->mx()) return block_body_mx(ctx, l, mod, n, s);
-  const h3dit_block_weights &w = ctx->blocks[l];
   const int D = ctx->cfg.hidden, I = ctx->inner(), F = ctx->cfg.ffn;
   const float *sh1 = mod, *sc1 = mod + D, *g1 = mod + 2 * D;
   const float *sh2 = mod + 3 * D, *sc2 = mod + 4 * D, *g2 = mod + 5 * D;
@@ -567,6 +624,101 @@ h3dit_status block_body(h3dit_ctx *ctx, int l, const float *mod, int n, cudaStre
     return st;
   return run_linear(ctx, H3DIT_EPI_GATED_RESIDUAL, ctx->u(), w.w_ff2, n, D, F, ctx->resid(), D, g2,
                     nullptr, s);
+}
+
+// AdaLN projections of the blocks in [l0, l1) whose weights are on the
+// device, one launch per run of consecutive such blocks (one launch per step
+// when every block is resident); streamed blocks get theirs from their slot.
+h3dit_status adaln_resident(h3dit_ctx *ctx, int l0, int l1, cudaStream_t s) {
+  int l = l0;
+  while (l < l1) {
+    if (ctx->streamed[l]) {
+      ++l;
+      continue;
+    }
+    int e = l;
+    while (e < l1 && !ctx->streamed[e]) ++e;
+    Launch L(ctx, H3DIT_KERNEL_ADALN, s);
+    h3dit_status st = ctx->cuda(launch_adaln(ctx->cvec(), ctx->wptr(), ctx->bptr(), l, e - l,
+                                             ctx->mod(l), ctx->cfg.hidden, ctx->num_sms, s),
+                                "adaln launch");
+    if (st) return st;
+    l = e;
+  }
+  return H3DIT_OK;
+}
+
+// Host weights of block l into staging slot `slot` on the copy stream, then
+// mark the slot ready (one cudaMemcpyAsync per weight tensor).
+h3dit_status copy_block(h3dit_ctx *ctx, int l, int slot) {
+  const h3dit_block_weights &w = ctx->blocks[l];
+  const void *src[6] = {w.w_qkv, w.w_o, w.w_ff1, w.w_ff2, w.w_ada, w.b_ada};
+  uint8_t *dst = ctx->staging + static_cast<size_t>(slot) * ctx->SP.slot;
+  for (int i = 0; i < 6; ++i) {
+    cudaError_t e = cudaMemcpyAsync(dst + ctx->SP.part[i], src[i], ctx->SP.bytes[i],
+                                    cudaMemcpyHostToDevice, ctx->copy);
+    if (e != cudaSuccess) return ctx->cuda(e, "weight streaming copy");
+  }
+  return ctx->cuda(cudaEventRecord(ctx->ready[slot], ctx->copy), "weight streaming event");
+}
+
+// Blocks [l0, l1) on the packed residual of n tokens. Resident blocks run on
+// their own weights with the modulation already in mod(l) (or `mod_one` for
+// a single block); a streamed block waits for its slot, gets its AdaLN
+// projection from the slot (unless `mod_one` is given) and runs on the slot.
+// Two slots alternate: the copy of streamed block i+2 starts on the copy
+// stream as soon as block i has finished with the slot, so it overlaps the
+// compute of block i+1. The copy stream forks from `s` at entry and joins it
+// at exit, so the whole call is ordered on `s` (and can be graph-captured).
+h3dit_status run_blocks(h3dit_ctx *ctx, int l0, int l1, int n, cudaStream_t s,
+                        const float *mod_one = nullptr) {
+  auto mod_of = [&](int l) { return mod_one ? mod_one : ctx->mod(l); };
+  std::vector<int> order;
+  for (int l = l0; l < l1; ++l)
+    if (ctx->streamed[l]) order.push_back(l);
+  h3dit_status st;
+  if (order.empty()) {
+    for (int l = l0; l < l1; ++l)
+      if ((st = block_body(ctx, l, ctx->blocks[l], mod_of(l), n, s))) return st;
+    return H3DIT_OK;
+  }
+  if (!ctx->staging)
+    return ctx->fail(H3DIT_ERR_WORKSPACE,
+                     "blocks with host weights need staging memory (h3dit_attach_staging)");
+  if ((st = ctx->cuda(cudaEventRecord(ctx->fork, s), "fork event"))) return st;
+  if ((st = ctx->cuda(cudaStreamWaitEvent(ctx->copy, ctx->fork, 0), "fork wait"))) return st;
+  const int first = static_cast<int>(order.size()) < 2 ? static_cast<int>(order.size()) : 2;
+  for (int i = 0; i < first; ++i)
+    if ((st = copy_block(ctx, order[i], i))) return st;
+  size_t i = 0;
+  for (int l = l0; l < l1; ++l) {
+    if (!ctx->streamed[l]) {
+      if ((st = block_body(ctx, l, ctx->blocks[l], mod_of(l), n, s))) return st;
+      continue;
+    }
+    const int slot = static_cast<int>(i % 2);
+    if ((st = ctx->cuda(cudaStreamWaitEvent(s, ctx->ready[slot], 0), "slot wait"))) return st;
+    if (!mod_one) {
+      const void *const *wt = reinterpret_cast<const void *const *>(ctx->staging + ctx->SP.table);
+      const float *const *bt =
+          reinterpret_cast<const float *const *>(ctx->staging + ctx->SP.table + 2 * sizeof(void *));
+      Launch L(ctx, H3DIT_KERNEL_ADALN, s);
+      if ((st = ctx->cuda(launch_adaln(ctx->cvec(), wt, bt, slot, 1, ctx->mod(l), ctx->cfg.hidden,
+                                       ctx->num_sms, s),
+                          "adaln launch")))
+        return st;
+    }
+    if ((st = block_body(ctx, l, ctx->slot_weights(slot), mod_of(l), n, s))) return st;
+    if (i + 2 < order.size()) {
+      if ((st = ctx->cuda(cudaEventRecord(ctx->slot_free[slot], s), "slot event"))) return st;
+      if ((st = ctx->cuda(cudaStreamWaitEvent(ctx->copy, ctx->slot_free[slot], 0), "slot wait")))
+        return st;
+      if ((st = copy_block(ctx, order[i + 2], slot))) return st;
+    }
+    ++i;
+  }
+  if ((st = ctx->cuda(cudaEventRecord(ctx->join, ctx->copy), "join event"))) return st;
+  return ctx->cuda(cudaStreamWaitEvent(s, ctx->join, 0), "join wait");
 }
 
 }  // namespace
@@ -639,6 +791,36 @@ h3dit_status h3dit_create(const h3dit_config *cfg, const h3dit_time_weights *tim
     delete ctx;
     return H3DIT_ERR_CUDA;
   }
+  // where each block's weights live: all on the device, or all in pinned
+  // host memory (streamed layer by layer through staging slots)
+  ctx->streamed.assign(cfg->n_blocks, 0);
+  for (int l = 0; l < cfg->n_blocks; ++l) {
+    const h3dit_block_weights &b = blocks[l];
+    const void *ptrs[6] = {b.w_qkv, b.w_o, b.w_ff1, b.w_ff2, b.w_ada, b.b_ada};
+    int host = 0, device = 0;
+    for (const void *p : ptrs) {
+      cudaPointerAttributes a{};
+      if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        a.type = cudaMemoryTypeUnregistered;
+      }
+      if (a.type == cudaMemoryTypeHost)
+        ++host;
+      else if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged)
+        ++device;
+    }
+    if (host == 6) {
+      ctx->streamed[l] = 1;
+      ++ctx->n_streamed;
+    } else if (device != 6) {
+      delete ctx;
+      return H3DIT_ERR_INVALID_ARG;  // mixed, or pageable host memory
+    }
+  }
+  if (ctx->n_streamed && ctx->mx()) {
+    delete ctx;
+    return H3DIT_ERR_UNSUPPORTED;  // MXFP8 quantizes every block at create
+  }
   std::vector<const void *> wp(cfg->n_blocks), bp(cfg->n_blocks);
   for (int l = 0; l < cfg->n_blocks; ++l) {
     wp[l] = blocks[l].w_ada;
@@ -687,6 +869,48 @@ h3dit_status h3dit_create(const h3dit_config *cfg, const h3dit_time_weights *tim
 }
 
 void h3dit_destroy(h3dit_ctx *ctx) { delete ctx; }
+
+size_t h3dit_staging_bytes(const h3dit_config *cfg) {
+  if (!config_ok(cfg)) return 0;
+  return staging_plan(cfg).total;
+}
+
+int32_t h3dit_streamed_blocks(const h3dit_ctx *ctx) { return ctx ? ctx->n_streamed : -1; }
+
+h3dit_status h3dit_attach_staging(h3dit_ctx *ctx, void *staging, size_t bytes, void *copy_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  const Staging S = staging_plan(&ctx->cfg);
+  if (!staging || (reinterpret_cast<uintptr_t>(staging) % kAlign) || bytes < S.total)
+    return ctx->fail(H3DIT_ERR_WORKSPACE, "staging needs %zu bytes, 256-byte aligned", S.total);
+  ctx->release_streaming();
+  ctx->SP = S;
+  ctx->staging = static_cast<uint8_t *>(staging);
+  cudaError_t e = cudaSuccess;
+  if (copy_stream) {
+    ctx->copy = static_cast<cudaStream_t>(copy_stream);
+  } else {
+    e = cudaStreamCreateWithFlags(&ctx->copy, cudaStreamNonBlocking);
+    ctx->own_copy = e == cudaSuccess;
+  }
+  for (cudaEvent_t *ev : {&ctx->fork, &ctx->join, &ctx->ready[0], &ctx->ready[1],
+                          &ctx->slot_free[0], &ctx->slot_free[1]})
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+  if (e == cudaSuccess) {
+    // the AdaLN kernel's pointer table for the two slots: w_ada[2], b_ada[2]
+    const void *table[4];
+    for (int s = 0; s < 2; ++s) {
+      const h3dit_block_weights w = ctx->slot_weights(s);
+      table[s] = w.w_ada;
+      table[2 + s] = w.b_ada;
+    }
+    e = cudaMemcpy(ctx->staging + S.table, table, sizeof(table), cudaMemcpyHostToDevice);
+  }
+  if (e != cudaSuccess) {
+    ctx->release_streaming();
+    return ctx->cuda(e, "attach staging");
+  }
+  return H3DIT_OK;
+}
 
 h3dit_status h3dit_sync_status(h3dit_ctx *ctx, void *cuda_stream) {
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
@@ -835,6 +1059,52 @@ h3dit_status h3dit_attention(h3dit_ctx *ctx, const void *q, const void *k, const
   return run_attention(ctx, q, k, v, ld_qkv, o, ld_o, n, static_cast<cudaStream_t>(cuda_stream));
 }
 
+h3dit_status h3dit_attention_heads(h3dit_ctx *ctx, int32_t heads, const void *q, const void *k,
+                                   const void *v, int32_t ld_qkv, void *o, int32_t ld_o, int32_t n,
+                                   void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (heads < 1) return ctx->fail(H3DIT_ERR_INVALID_ARG, "heads < 1");
+  return run_attention(ctx, q, k, v, ld_qkv, o, ld_o, n, static_cast<cudaStream_t>(cuda_stream),
+                       nullptr, heads);
+}
+
+namespace {
+h3dit_status check_sp(h3dit_ctx *ctx, const void *a, const void *b, int n_local, int ranks) {
+  if (!a || !b || !aligned16(a) || !aligned16(b))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "sequence parallel re-layout: NULL or misaligned pointer");
+  if (n_local < 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "n_local < 0");
+  if (ranks < 1 || ctx->cfg.heads % ranks)
+    return ctx->fail(H3DIT_ERR_UNSUPPORTED, "%d ranks do not divide %d heads", ranks, ctx->cfg.heads);
+  if ((ctx->inner() / ranks) % 8)
+    return ctx->fail(H3DIT_ERR_UNSUPPORTED, "a head group's width is not a multiple of 8");
+  return H3DIT_OK;
+}
+}  // namespace
+
+h3dit_status h3dit_sp_pack_qkv(h3dit_ctx *ctx, const void *qkv, int32_t n_local, int32_t ranks,
+                               void *send, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  h3dit_status st = check_sp(ctx, qkv, send, n_local, ranks);
+  if (st || n_local == 0) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  Launch L(ctx, H3DIT_KERNEL_PACK, s);
+  return ctx->cuda(launch_sp_pack_qkv(qkv, n_local, ranks, ctx->inner() / ranks, send,
+                                      ctx->num_sms, s),
+                   "sequence parallel pack launch");
+}
+
+h3dit_status h3dit_sp_unpack_o(h3dit_ctx *ctx, const void *recv, int32_t n_local, int32_t ranks,
+                               void *o, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  h3dit_status st = check_sp(ctx, recv, o, n_local, ranks);
+  if (st || n_local == 0) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  Launch L(ctx, H3DIT_KERNEL_PACK, s);
+  return ctx->cuda(launch_sp_unpack_o(recv, n_local, ranks, ctx->inner() / ranks, o, ctx->num_sms,
+                                      s),
+                   "sequence parallel unpack launch");
+}
+
 h3dit_status h3dit_block_forward(h3dit_ctx *ctx, int32_t block, float t, const float *mod,
                                  void *x_img, const h3dit_grid *grids, int32_t n_grids,
                                  void *x_txt, int32_t n_txt, void *cuda_stream) {
@@ -850,11 +1120,10 @@ h3dit_status h3dit_block_forward(h3dit_ctx *ctx, int32_t block, float t, const f
   if ((st = rope_table_into(ctx, grids, n_grids, n_txt, n, ctx->rope(), s))) return st;
   if (!mod) {
     if ((st = h3dit_time_embed(ctx, t, ctx->cvec(), s))) return st;
-    if ((st = h3dit_adaln_project(ctx, ctx->cvec(), block, 1, ctx->mod(block), s))) return st;
-    mod = ctx->mod(block);
+    if ((st = adaln_resident(ctx, block, block + 1, s))) return st;
   }
   if ((st = run_pack(ctx, x_txt, n_txt, x_img, n_img, s))) return st;
-  if ((st = block_body(ctx, block, mod, n, s))) return st;
+  if ((st = run_blocks(ctx, block, block + 1, n, s, mod))) return st;
   return run_unpack(ctx, n_txt, n_img, x_txt, x_img, s);
 }
 
@@ -868,10 +1137,9 @@ h3dit_status h3dit_step(h3dit_ctx *ctx, float t, void *x_img, const h3dit_grid *
   const int n = n_txt + n_img;
   if ((st = rope_table_into(ctx, grids, n_grids, n_txt, n, ctx->rope(), s))) return st;
   if ((st = h3dit_time_embed(ctx, t, ctx->cvec(), s))) return st;
-  if ((st = h3dit_adaln_project(ctx, ctx->cvec(), 0, ctx->cfg.n_blocks, ctx->mod(0), s))) return st;
+  if ((st = adaln_resident(ctx, 0, ctx->cfg.n_blocks, s))) return st;
   if ((st = run_pack(ctx, x_txt, n_txt, x_img, n_img, s))) return st;
-  for (int l = 0; l < ctx->cfg.n_blocks; ++l)
-    if ((st = block_body(ctx, l, ctx->mod(l), n, s))) return st;
+  if ((st = run_blocks(ctx, 0, ctx->cfg.n_blocks, n, s))) return st;
   return run_unpack(ctx, n_txt, n_img, x_txt, x_img, s);
 }
 
@@ -907,7 +1175,7 @@ h3dit_status h3dit_denoise(h3dit_ctx *ctx, const h3dit_io_weights *io, float *la
     const double tn = 1.0 - static_cast<double>(k + 1) / n_steps;
     const float t = static_cast<float>(tk);
     if ((st = h3dit_time_embed(ctx, t, ctx->cvec(), s))) return st;
-    if ((st = h3dit_adaln_project(ctx, ctx->cvec(), 0, ctx->cfg.n_blocks, ctx->mod(0), s))) return st;
+    if ((st = adaln_resident(ctx, 0, ctx->cfg.n_blocks, s))) return st;
     {
       Launch L(ctx, H3DIT_KERNEL_IO, s);
       if ((st = ctx->cuda(launch_output_modulation(ctx->cvec(), io->w_mod, io->b_mod, ctx->omod(),
@@ -923,8 +1191,7 @@ h3dit_status h3dit_denoise(h3dit_ctx *ctx, const h3dit_io_weights *io, float *la
                           "embed latent launch")))
         return st;
     }
-    for (int l = 0; l < ctx->cfg.n_blocks; ++l)
-      if ((st = block_body(ctx, l, ctx->mod(l), static_cast<int>(n), s))) return st;
+    if ((st = run_blocks(ctx, 0, ctx->cfg.n_blocks, static_cast<int>(n), s))) return st;
     Launch L(ctx, H3DIT_KERNEL_IO, s, 2);
     if ((st = ctx->cuda(launch_output_euler(x_img, true, ctx->omod(), io->w_out, io->b_out, D,
                                             ctx->cfg.norm_eps, latent, channels, lat_h, lat_w,

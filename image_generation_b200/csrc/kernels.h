@@ -155,6 +155,12 @@ cudaError_t launch_output_modulation(const float *c, const float *w_mod, const f
 cudaError_t launch_output_euler(const void *x, bool in_fp32, const float *mod, const float *w_out,
                                 const float *b_out, int D, float eps, float *z, int C, int Hl,
                                 int Wl, float dt, float *rinv_scratch, cudaStream_t s);
+// Ulysses sequence parallelism (sp.cu): the re-layouts around the two
+// all-to-alls; cw = columns of one head group per matrix (I / ranks).
+cudaError_t launch_sp_pack_qkv(const void *qkv, int n, int ranks, int cw, void *send, int num_sms,
+                               cudaStream_t s);
+cudaError_t launch_sp_unpack_o(const void *recv, int n, int ranks, int cw, void *o, int num_sms,
+                               cudaStream_t s);
 cudaError_t launch_mx_tile_sf(const uint8_t *sf, int n, int k, uint8_t *tiled, cudaStream_t s);
 // bf16 [rows, k] (row stride ld elements) -> E4M3 [rows, k] + scales.
 cudaError_t launch_mx_quantize(const void *src, long long ld, int rows, int k, uint8_t *dst,

@@ -110,6 +110,12 @@ def _load() -> C.CDLL:
         "h3dit_output_euler": (i32, [p, p, p, p, p, p, i32, i32, i32, f32, p]),
         "h3dit_denoise": (i32, [p, C.POINTER(h3dit_io_weights), p, i32, i32, i32, p, i32, i32,
                                 p]),
+        "h3dit_attention_heads": (i32, [p, i32, p, p, p, i32, p, i32, i32, p]),
+        "h3dit_sp_pack_qkv": (i32, [p, p, i32, i32, p, p]),
+        "h3dit_sp_unpack_o": (i32, [p, p, i32, i32, p, p]),
+        "h3dit_staging_bytes": (sz, [C.POINTER(h3dit_config)]),
+        "h3dit_attach_staging": (i32, [p, p, sz, p]),
+        "h3dit_streamed_blocks": (i32, [p]),
         "h3dit_selftest_bounded_wait": (i32, [p, i32, p]),
         "h3dit_profile_begin": (i32, [p]),
         "h3dit_profile_end": (i32, [p, C.POINTER(C.c_float), C.POINTER(C.c_int64)]),
@@ -190,6 +196,16 @@ def _ptr(t, dense: bool = True) -> int | None:
     return t.data_ptr()
 
 
+def _wptr(t) -> int:
+    """Address of a block weight: a contiguous CUDA tensor, or a contiguous
+    pinned host tensor (a block the library streams to the GPU)."""
+    if not t.is_cuda and not t.is_pinned():
+        raise H3DitError(H3DIT_ERR_INVALID_ARG, "host weights must be in pinned memory")
+    if not t.is_contiguous():
+        raise H3DitError(H3DIT_ERR_INVALID_ARG, "tensor argument is not contiguous")
+    return t.data_ptr()
+
+
 def _stream(stream=None) -> int:
     import torch
 
@@ -221,13 +237,29 @@ class Context:
                                 _ptr(time_w["w_t2"]), _ptr(time_w["b_t2"]))
         arr = (h3dit_block_weights * len(blocks))()
         for i, b in enumerate(blocks):
-            arr[i] = h3dit_block_weights(_ptr(b["w_qkv"]), _ptr(b["w_o"]), _ptr(b["w_ff1"]),
-                                         _ptr(b["w_ff2"]), _ptr(b["w_ada"]), _ptr(b["b_ada"]))
+            arr[i] = h3dit_block_weights(_wptr(b["w_qkv"]), _wptr(b["w_o"]), _wptr(b["w_ff1"]),
+                                         _wptr(b["w_ff2"]), _wptr(b["w_ada"]), _wptr(b["b_ada"]))
         handle = C.c_void_p()
         st = lib.h3dit_create(C.byref(cfg), C.byref(tw), arr, _ptr(self.workspace),
                               ws_bytes, _stream(stream), C.byref(handle))
         check(None, st)
         self.handle = handle
+
+    def attach_staging(self, staging=None, copy_stream=None) -> None:
+        """Lend the context device staging memory for blocks whose weights are
+        in pinned host memory (allocated here when omitted)."""
+        import torch
+
+        nbytes = int(lib.h3dit_staging_bytes(C.byref(self.cfg)))
+        if staging is None:
+            staging = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        self.staging = staging
+        self._check(lib.h3dit_attach_staging(self.handle, _ptr(staging),
+                                             staging.numel() * staging.element_size(),
+                                             None if copy_stream is None else copy_stream.cuda_stream))
+
+    def streamed_blocks(self) -> int:
+        return int(lib.h3dit_streamed_blocks(self.handle))
 
     def close(self) -> None:
         if getattr(self, "handle", None):
@@ -269,6 +301,30 @@ class Context:
         self._check(lib.h3dit_attention(self.handle, _ptr(q, False), _ptr(k, False),
                                         _ptr(v, False), ld_qkv, _ptr(o, False), ld_o, n,
                                         _stream(stream)))
+
+    def empty(self, shape, kind: str):
+        """A device buffer for the sequence-parallel driver: "act" is bf16
+        (token-major activations), "f32" and "rope" are fp32."""
+        import torch
+
+        dt = torch.bfloat16 if kind == "act" else torch.float32
+        return torch.empty(*shape, dtype=dt, device="cuda")
+
+    def attention_heads(self, heads: int, q, k, v, ld_qkv: int, o, ld_o: int, n: int,
+                        stream=None) -> None:
+        self._check(lib.h3dit_attention_heads(self.handle, heads, _ptr(q, False), _ptr(k, False),
+                                              _ptr(v, False), ld_qkv, _ptr(o, False), ld_o, n,
+                                              _stream(stream)))
+
+    def sp_pack_qkv(self, qkv, ranks: int, send, stream=None) -> None:
+        """qkv [n_local, 3I] -> send [ranks][n_local][3I/ranks] (head groups)."""
+        self._check(lib.h3dit_sp_pack_qkv(self.handle, _ptr(qkv), qkv.shape[0], ranks, _ptr(send),
+                                          _stream(stream)))
+
+    def sp_unpack_o(self, recv, ranks: int, o, stream=None) -> None:
+        """recv [ranks][n_local][I/ranks] -> o [n_local, I]."""
+        self._check(lib.h3dit_sp_unpack_o(self.handle, _ptr(recv), o.shape[0], ranks, _ptr(o),
+                                          _stream(stream)))
 
     def block_forward(self, block: int, t: float, x_img, grids, x_txt, mod=None,
                       stream=None) -> None:

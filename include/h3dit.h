@@ -114,19 +114,55 @@ const char *h3dit_last_error(const h3dit_ctx *ctx);
  * scales repacked for 224-column tiles where N is a multiple of 224). */
 size_t h3dit_workspace_bytes(const h3dit_config *cfg);
 
-/* Create a context. `blocks` points to cfg->n_blocks host structs whose device
- * pointers must stay valid until h3dit_destroy. `workspace` is device memory of
- * at least h3dit_workspace_bytes(cfg) bytes, 256-byte aligned, lent to the
- * context for its life. Copies the weight pointer table to the device and,
- * with H3DIT_PRECISION_MXFP8, quantizes every block's linears, on
- * `cuda_stream`, then synchronises that stream once before returning (the
- * host-side table must have been consumed). On error *out is set to NULL. */
+/* Create a context. `blocks` points to cfg->n_blocks host structs whose
+ * pointers must stay valid until h3dit_destroy. Each block's six weight
+ * pointers are either all device memory or all pinned host memory
+ * (cudaHostAlloc / cudaHostRegister, e.g. torch's pin_memory); host blocks are
+ * streamed to the GPU layer by layer (see h3dit_attach_staging); pageable host
+ * memory or a mix within one block is H3DIT_ERR_INVALID_ARG, and host blocks
+ * with H3DIT_PRECISION_MXFP8 are H3DIT_ERR_UNSUPPORTED. The timestep weights
+ * are device memory. `workspace` is device memory of at least
+ * h3dit_workspace_bytes(cfg) bytes, 256-byte aligned, lent to the context for
+ * its life. Copies the weight pointer table to the device and, with
+ * H3DIT_PRECISION_MXFP8, quantizes every block's linears, on `cuda_stream`,
+ * then synchronises that stream once before returning (the host-side table
+ * must have been consumed). On error *out is set to NULL. */
 h3dit_status h3dit_create(const h3dit_config *cfg, const h3dit_time_weights *time_w,
                           const h3dit_block_weights *blocks, void *workspace, size_t ws_bytes,
                           void *cuda_stream, h3dit_ctx **out);
 
 /* Frees the host state of a context (NULL-safe). Device memory is the caller's. */
 void h3dit_destroy(h3dit_ctx *ctx);
+
+/* ---- Layerwise weight streaming ------------------------------------------
+ * "H3-Image Day-0 Support: 4K in 0.87s with Vera Rubin", "Fitting Smaller
+ * GPUs", and the vLLM-Omni recipe's "Deployment profiles" (DLO): the DiT's
+ * blocks stay in pinned host memory and move to the GPU one block at a time.
+ * Here a context whose blocks are partly or wholly in pinned host memory
+ * copies each such block's six weight tensors (one cudaMemcpyAsync each) into
+ * one of two device staging slots on a copy stream. The slots alternate: the
+ * copy of the next-but-one host block starts as soon as a block has finished
+ * with its slot, so it overlaps the block in between. Device-resident blocks
+ * run as usual (their AdaLN projections still in one launch per step); a
+ * host block's AdaLN projection is computed from its slot just before it
+ * runs. Results are bit-identical to the same weights held on the device.
+ * Every call is still ordered on its `cuda_stream`: the copy stream forks
+ * from it at entry and joins it at exit (so a step can be graph-captured). */
+
+/* Bytes of staging memory h3dit_attach_staging needs for `cfg` (two slots of
+ * one block's weights and a small pointer table), or 0 if `cfg` is invalid. */
+size_t h3dit_staging_bytes(const h3dit_config *cfg);
+
+/* Lend the context `staging`, device memory of at least
+ * h3dit_staging_bytes(&cfg) bytes, 256-byte aligned, for its life (or until
+ * the next attach), and the stream the weight copies run on: `copy_stream`,
+ * or a stream the context creates (and destroys) when it is NULL. Writes the
+ * slots' pointer table with one synchronous copy. Without staging, a call
+ * that runs a host block returns H3DIT_ERR_WORKSPACE before enqueuing it. */
+h3dit_status h3dit_attach_staging(h3dit_ctx *ctx, void *staging, size_t bytes, void *copy_stream);
+
+/* Number of blocks whose weights are in host memory (-1 for a NULL ctx). */
+int32_t h3dit_streamed_blocks(const h3dit_ctx *ctx);
 
 /* Run block `block` in place on the packed sequence [x_txt; images]:
  *   x_txt  device [n_txt, D] (may be NULL when n_txt == 0), in/out;
@@ -195,6 +231,40 @@ h3dit_status h3dit_linear(h3dit_ctx *ctx, int32_t epilogue, const void *a, const
 h3dit_status h3dit_attention(h3dit_ctx *ctx, const void *q, const void *k, const void *v,
                              int32_t ld_qkv, void *o, int32_t ld_o, int32_t n,
                              void *cuda_stream);
+
+/* ---- Ulysses sequence parallelism over P ranks -------------------------
+ * "H3-Image Day-0 Support: 4K in 0.87s with Vera Rubin", "Faster DiT"
+ * (Ulysses SP4) and the vLLM-Omni recipe's "Deployment profiles" (SP 2,
+ * SP 4). Each of P ranks holds n_local = N / P consecutive tokens of the
+ * packed sequence and runs every step of the block but the attention on
+ * them, with all heads. Around the attention two all-to-alls (NCCL, by the
+ * caller) trade that for all N tokens and heads / P: the re-layouts on either
+ * side are below, and h3dit_attention_heads runs the attention on the head
+ * group. ranks must divide cfg->heads, and heads*head_dim/ranks must be a
+ * multiple of 8. */
+
+/* a5 for `heads` (1 .. cfg->heads) heads: as h3dit_attention with the heads
+ * count given instead of cfg->heads (o gets heads*head_dim columns). */
+h3dit_status h3dit_attention_heads(h3dit_ctx *ctx, int32_t heads, const void *q, const void *k,
+                                   const void *v, int32_t ld_qkv, void *o, int32_t ld_o, int32_t n,
+                                   void *cuda_stream);
+
+/* Before the first all-to-all: qkv device bf16 [n_local, 3I] (this rank's
+ * tokens, the QKV step's output) -> send device bf16 [ranks][n_local][3I/ranks]
+ * (dense), where block d holds, for each row, the Q | K | V columns of heads
+ * d*H/ranks .. (d+1)*H/ranks - 1. Sent block d to rank d, the receive buffer
+ * [ranks][n_local][3I/ranks] of rank d is the Q|K|V matrix of its heads for
+ * all tokens in sequence order, for h3dit_attention_heads with heads = H/ranks
+ * and ld_qkv = 3I/ranks. */
+h3dit_status h3dit_sp_pack_qkv(h3dit_ctx *ctx, const void *qkv, int32_t n_local, int32_t ranks,
+                               void *send, void *cuda_stream);
+
+/* After the second all-to-all (the attention output [N, I/ranks] of this
+ * rank's heads sent in row blocks of n_local): recv device bf16
+ * [ranks][n_local][I/ranks], block s from head group s -> o device bf16
+ * [n_local, I] with head group s at columns s*I/ranks .. (s+1)*I/ranks - 1. */
+h3dit_status h3dit_sp_unpack_o(h3dit_ctx *ctx, const void *recv, int32_t n_local, int32_t ranks,
+                               void *o, void *cuda_stream);
 
 /* ---- a11: the MXFP8 variant of the four block linears ------------------
  * "H3-Image Day-0 Support: 4K in 0.87s with Vera Rubin", "Faster DiT" and

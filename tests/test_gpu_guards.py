@@ -101,9 +101,9 @@ def test_linear_epilogues(bf16_ctx, m):
     out.check(f"QKV + RoPE, m={m}")
     x = Guarded((m, D), torch.float32, init=torch.randn(m, D, device="cuda"))
     gate = torch.full((D,), 0.25, device="cuda")
-    wo = to_dev(synth.normal_bf16((D, 800), 0.02, m, "wo"))
-    a800 = to_dev(synth.tokens(m, 800, m, "a800"))
-    ctx.linear(H.H3DIT_EPI_GATED_RESIDUAL, a800, wo, x.t, gate=gate)
+    wo = to_dev(synth.normal_bf16((D, 832), 0.02, m, "wo"))   # k = 13 k-blocks of 64
+    a832 = to_dev(synth.tokens(m, 832, m, "a832"))
+    ctx.linear(H.H3DIT_EPI_GATED_RESIDUAL, a832, wo, x.t, gate=gate)
     x.check(f"gated residual, m={m}")
     _ok(ctx, ws, f"linear m={m}")
 

@@ -1,0 +1,117 @@
+"""Ulysses sequence parallelism on the GPU path, with P ranks emulated in one
+process on one GPU: each rank's stages run libh3dit's kernels through
+image_generation_b200.ulysses (RMSNorm, QKV + RoPE on its rows, the head-group
+re-layouts, attention on its head group, out-projection and FFN), and the two
+all-to-alls are done by device copies between the ranks' buffers - the same
+data movement NCCL's all_to_all_single does between GPUs. No kernel waits on
+another rank. Every kernel computes each output element the same way whatever
+rows or heads it is given, so the result must equal the unsharded step bit
+for bit."""
+import pytest
+
+from image_generation_b200 import synth
+from tests.helpers import block_tensors, time_tensors
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+def _exchange_qkv(ranks):
+    P = len(ranks)
+    for d in range(P):
+        for s in range(P):
+            ranks[d].recv1[s].copy_(ranks[s].send1[d])
+
+
+def _exchange_o(ranks):
+    P = len(ranks)
+    n = ranks[0].n
+    for d in range(P):
+        for s in range(P):
+            ranks[d].recv2[s].copy_(ranks[s].o_heads[d * n:(d + 1) * n])
+
+
+def _emulated_step(ctx, weights, P, dims, t, x, grids, n_txt):
+    from image_generation_b200.ulysses import UlyssesRank
+
+    n_total = x.shape[0]
+    ranks = [UlyssesRank(ctx, r, P, n_total, dims.hidden, dims.heads, dims.head_dim, dims.ffn)
+             for r in range(P)]
+    c = torch.empty(dims.hidden, device="cuda")
+    mod = torch.empty(len(weights), 6, dims.hidden, device="cuda")
+    rope = torch.empty(n_total, dims.head_dim // 2, 2, device="cuda")
+    ctx.time_embed(t, c)
+    ctx.adaln_project(c, 0, len(weights), mod)
+    ctx.rope_table(grids, n_txt, rope)
+    xs = [x[r.rows()].clone() for r in ranks]
+    for l, w in enumerate(weights):
+        for i, r in enumerate(ranks):
+            r.qkv_and_pack(xs[i], mod[l], w, rope[r.rows()])
+        _exchange_qkv(ranks)
+        for r in ranks:
+            r.attention()
+        _exchange_o(ranks)
+        for i, r in enumerate(ranks):
+            r.finish(xs[i], mod[l], w)
+    return torch.cat(xs)
+
+
+def _run(dims, n_blocks, P, n_txt, grids, seed):
+    from image_generation_b200 import h3dit as H
+
+    tw = time_tensors(synth.time_weights(dims, seed))
+    weights = [block_tensors(synth.block_weights(dims, seed + 100 + l)) for l in range(n_blocks)]
+    n_total = n_txt + sum(h * w for _, h, w in grids)
+    cfg = H.make_config(dims.hidden, dims.heads, dims.head_dim, dims.ffn, n_blocks, n_total,
+                        io_fp32=True)
+    ctx = H.Context(cfg, tw, weights)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    x = torch.randn(n_total, dims.hidden, device="cuda", generator=g)
+    got = _emulated_step(ctx, weights, P, dims, 0.4, x, grids, n_txt)
+    xt, xi = x[:n_txt].clone(), x[n_txt:].clone()
+    ctx.step(0.4, xi, grids, xt)
+    torch.cuda.synchronize()
+    assert ctx.sync_status() == 0
+    ref = torch.cat([xt, xi])
+    assert not torch.equal(ref, x)
+    return got, ref
+
+
+@pytest.mark.parametrize("P", [2, 4, 8])
+def test_emulated_ranks_small(P):
+    got, ref = _run(synth.SMALL, 2, P, 32, [(0, 16, 16)], 1)
+    assert torch.equal(got, ref), f"max diff {float((got - ref).abs().max())}"
+
+
+def test_emulated_ranks_head_dim_128():
+    dims = synth.Dims(hidden=768, heads=8, head_dim=128, ffn=2048)
+    got, ref = _run(dims, 2, 4, 8, [(0, 12, 20), (1, 4, 4)], 2)
+    assert torch.equal(got, ref), f"max diff {float((got - ref).abs().max())}"
+
+
+@pytest.mark.parametrize("P", [4, 8])
+def test_emulated_ranks_full_width_4096(P):
+    """SP4 and SP8 at full width on the 4096^2 sequence (16,896 tokens, 14 and 7
+    heads per rank), one block."""
+    got, ref = _run(synth.FULL_96, 1, P, 512, [(0, 128, 128)], 3)
+    assert torch.equal(got, ref), f"max diff {float((got - ref).abs().max())}"
+
+
+def test_relayout_errors():
+    from image_generation_b200 import h3dit as H
+
+    dims = synth.SMALL
+    cfg = H.make_config(dims.hidden, dims.heads, dims.head_dim, dims.ffn, 1, 64)
+    ctx = H.Context(cfg, time_tensors(synth.time_weights(dims, 0)),
+                    [block_tensors(synth.block_weights(dims, 0))])
+    qkv = torch.zeros(16, 3 * dims.inner, device="cuda", dtype=torch.bfloat16)
+    send = torch.zeros(3, 16, dims.inner, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(H.H3DitError) as e:   # 3 ranks do not divide 8 heads
+        ctx.sp_pack_qkv(qkv, 3, send)
+    assert e.value.status == H.H3DIT_ERR_UNSUPPORTED
+    with pytest.raises(H.H3DitError) as e:   # more heads than the context has
+        ctx.attention_heads(9, qkv, qkv, qkv, 3 * dims.inner, send.view(16, -1), 3 * dims.inner, 16)
+    assert e.value.status == H.H3DIT_ERR_INVALID_ARG
+    assert ctx.sync_status() == 0
