@@ -201,3 +201,48 @@ def ragged(dims: Dims, n_txt: int, grids: Sequence[Tuple[int, int, int]], seed: 
            t: float = 0.5, name: str = "ragged") -> Workload:
     """A workload with arbitrary token counts (for tails and edge cases)."""
     return Workload(name, dims, n_txt, tuple(tuple(g) for g in grids), seed, t)
+
+
+# --- the image VAE's ViT decoder (shape level) --------------------------------
+# The same recipe: linears N(0, 0.02) rounded to bf16 (the pages' BF16 decode
+# control), their biases and the LayerNorm gains and biases fp32, drawn
+# (gains 1 + N(0, 0.1), biases N(0, 0.02)) so that every affine term is
+# exercised. Latents N(0, 1) in fp32.
+
+@dataclasses.dataclass(frozen=True)
+class VaeDims:
+    width: int = 1280
+    heads: int = 10
+    head_dim: int = 128
+    mlp: int = 5120
+    layers: int = 24
+    tile: int = 32
+    channels: int = 24
+    out_features: int = 768  # 3 x 16 x 16 pixels per token
+
+
+VAE = VaeDims()
+VAE_SMALL = VaeDims(width=256, heads=2, head_dim=128, mlp=1024, layers=2, tile=16)
+
+
+def vae_weights(v: VaeDims, seed: int, std: float = 0.02) -> Dict:
+    """Random-init decoder weights, nn.Linear layout [out, in]; w_qkv rows are
+    [Q heads | K heads | V heads], each head's head_dim rows contiguous."""
+    W, M = v.width, v.mlp
+    f = lambda shape, tag, s=std: normal_f32(shape, s, seed, tag)
+    gain = lambda tag: (1.0 + normal_f32((W,), 0.1, seed, tag)).astype(np.float32)
+    layers = []
+    for l in range(v.layers):
+        t = f"l{l}_"
+        layers.append({
+            "ln1_g": gain(t + "ln1_g"), "ln1_b": f((W,), t + "ln1_b"),
+            "w_qkv": normal_bf16((3 * W, W), std, seed, t + "w_qkv"), "b_qkv": f((3 * W,), t + "b_qkv"),
+            "w_o": normal_bf16((W, W), std, seed, t + "w_o"), "b_o": f((W,), t + "b_o"),
+            "ln2_g": gain(t + "ln2_g"), "ln2_b": f((W,), t + "ln2_b"),
+            "w_1": normal_bf16((M, W), std, seed, t + "w_1"), "b_1": f((M,), t + "b_1"),
+            "w_2": normal_bf16((W, M), std, seed, t + "w_2"), "b_2": f((W,), t + "b_2"),
+        })
+    return {"w_in": normal_f32((W, v.channels), 0.2, seed, "w_in"), "b_in": f((W,), "b_in"),
+            "layers": layers, "lnf_g": gain("lnf_g"), "lnf_b": f((W,), "lnf_b"),
+            "w_out": normal_bf16((v.out_features, W), std, seed, "w_out"),
+            "b_out": f((v.out_features,), "b_out")}

@@ -8,23 +8,32 @@ if ROOT not in sys.path:
 # With H3_ORACLE_MUTANT set (only tests/test_oracle_mutations.py sets it, in a
 # child process), the oracle module is replaced by a copy with one planted
 # mistake from tests/oracle_mutants.py, so that the pins can be shown to catch it.
-_MUTANT = os.environ.get("H3_ORACLE_MUTANT")
-if _MUTANT:
+# H3_VAE_MUTANT does the same for oracle/vae_decoder.py.
+def _plant(module: str, table: dict, name: str) -> None:
     import types
 
     import oracle
+
+    _old, _new = table[name]
+    path = os.path.join(ROOT, "oracle", module + ".py")
+    with open(path) as fh:
+        src = fh.read()
+    assert _old in src, name
+    mod = types.ModuleType("oracle." + module)
+    mod.__file__ = path
+    sys.modules["oracle." + module] = mod
+    exec(compile(src.replace(_old, _new, 1), path, "exec"), mod.__dict__)
+    setattr(oracle, module, mod)
+
+
+if os.environ.get("H3_ORACLE_MUTANT"):
     from tests.oracle_mutants import MUTANTS
 
-    _old, _new = MUTANTS[_MUTANT]
-    _path = os.path.join(ROOT, "oracle", "dit_block.py")
-    with open(_path) as _fh:
-        _src = _fh.read()
-    assert _old in _src, _MUTANT
-    _mod = types.ModuleType("oracle.dit_block")
-    _mod.__file__ = _path
-    sys.modules["oracle.dit_block"] = _mod
-    exec(compile(_src.replace(_old, _new, 1), _path, "exec"), _mod.__dict__)
-    oracle.dit_block = _mod
+    _plant("dit_block", MUTANTS, os.environ["H3_ORACLE_MUTANT"])
+if os.environ.get("H3_VAE_MUTANT"):
+    from tests.oracle_mutants import VAE_MUTANTS
+
+    _plant("vae_decoder", VAE_MUTANTS, os.environ["H3_VAE_MUTANT"])
 
 
 def pytest_configure(config):
