@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-mxfp8", action="store_true")
+    ap.add_argument("--no-vae", action="store_true",
+                    help="skip the VAE decoder timing")
     ap.add_argument("--no-streaming", action="store_true",
                     help="skip the layerwise weight-streaming timings")
     ap.add_argument("--no-denoise", action="store_true",
@@ -648,6 +650,79 @@ def streaming_timings(tw, blocks, x_txt, x_img, grids, dh, residents=(24, 8), st
     return out
 
 
+def vae_flops(n_tok: int, tile: int, W=1280, M=5120, layers=24, C=24) -> float:
+    """Algorithmic flops of a decode: the linears per token, plus 4 n^2 W per
+    tile and layer for the attention over a tile's n tokens."""
+    n = tile * tile
+    lin = n_tok * (2 * C * W + layers * 2 * (4 * W * W + 2 * W * M) + 2 * W * 768)
+    return float(lin + layers * (n_tok // n) * 4 * n * n * W)
+
+
+def vae_timing(reps: int = 5) -> dict:
+    """The image VAE's 24-layer ViT decoder (width 1280, 10 heads x 128, MLP
+    5120, 32 x 32 latent tiles) decoding the 4096^2 canvas's latent
+    [24, 256, 256] (64 tiles, 65,536 tokens) on random device weights: ms per
+    decode eagerly and replayed from a CUDA graph, TFLOP/s, kernel shares."""
+    import torch
+
+    from image_generation_b200 import h3dit as Hb
+
+    W, M, L_, T = 1280, 5120, 24, 32
+    g = torch.Generator(device="cuda")
+    g.manual_seed(11)
+    mat = lambda *s: (torch.randn(*s, device="cuda", generator=g) * 0.02).bfloat16()
+    vec = lambda n, base=0.0: torch.randn(n, device="cuda", generator=g) * 0.02 + base
+    layers = [{"ln1_g": vec(W, 1.0), "ln1_b": vec(W), "w_qkv": mat(3 * W, W), "b_qkv": vec(3 * W),
+               "w_o": mat(W, W), "b_o": vec(W), "ln2_g": vec(W, 1.0), "ln2_b": vec(W),
+               "w_1": mat(M, W), "b_1": vec(M), "w_2": mat(W, M), "b_2": vec(W)}
+              for _ in range(L_)]
+    weights = {"w_in": torch.randn(W, 24, device="cuda", generator=g) * 0.2, "b_in": vec(W),
+               "layers": layers, "lnf_g": vec(W, 1.0), "lnf_b": vec(W), "w_out": mat(768, W),
+               "b_out": vec(768)}
+    hl = 2 * GRID  # latent side: 16x VAE downsampling of the 4096^2 canvas
+    cfg = Hb.make_vae_config(W, 10, 128, M, L_, T, 24, hl * hl)
+    dec = Hb.VaeDecoder(cfg, weights)
+    z = torch.randn(24, hl, hl, device="cuda", generator=g)
+    img = torch.empty(3, 16 * hl, 16 * hl, device="cuda")
+    for _ in range(2):
+        dec.decode(z, img)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dec.profile_begin()
+    e0.record()
+    for _ in range(reps):
+        dec.decode(z, img)
+    e1.record()
+    torch.cuda.synchronize()
+    prof = dec.profile_end()
+    ms = e0.elapsed_time(e1) / reps
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        dec.decode(z, img)
+    graph.replay()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    g_ms = e0.elapsed_time(e1) / reps
+    del graph
+    if dec.sync_status() != 0 or not bool(torch.isfinite(img).all()):
+        raise RuntimeError("VAE decode failed")
+    fl = vae_flops(hl * hl, T)
+    tot = sum(v[0] for v in prof.values()) or 1.0
+    att_ms, att_n = prof["attention"]
+    att_fl = L_ * (hl * hl // (T * T)) * 4.0 * (T * T) ** 2 * W
+    out = {"ms": round(ms, 2), "graph_ms": round(g_ms, 2), "tokens": hl * hl,
+           "tiles": hl * hl // (T * T), "image": [3, 16 * hl, 16 * hl],
+           "tflops": round(fl / ms / 1e9, 1),
+           "attention_tflops": round(att_fl * reps / att_ms / 1e9, 1) if att_n else None,
+           "kernel_share": {k: round(v[0] / tot, 4) for k, v in prof.items() if v[1]}}
+    dec.close()
+    return out
+
+
 def block_flops(n: int, d) -> float:
     I = d.heads * d.head_dim
     return 8.0 * n * d.hidden * I + 4.0 * n * d.hidden * d.ffn + 4.0 * n * n * I
@@ -811,6 +886,10 @@ def run_h3dit(args):
                            "d2h_bytes_per_run": h_out.numel() * 4}}
         del io, noise, lat
 
+    vae = None
+    if world == 1 and not args.no_vae:
+        vae = vae_timing()
+
     streaming = None
     if world == 1 and not args.no_streaming:
         streaming = streaming_timings(tw, blocks, x_txt, x_img, grids, dh)
@@ -870,6 +949,7 @@ def run_h3dit(args):
             "six_step_ms": round(6 * ms_step, 1),
             "denoise_6step": denoise,
             "weight_streaming": streaming,
+            "vae_decode_4096": vae,
             "graph_ms_per_step": None if graph_ms is None else round(graph_ms, 2),
         }
         gemm_kinds = ("qkv", "out_proj", "ffn1", "ffn2")

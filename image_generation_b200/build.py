@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libh3dit.so")
 SOURCES = ["api.cu", "gemm.cu", "gemm_pair.cu", "gemm_mx.cu", "attention.cu", "elementwise.cu",
-           "io_layers.cu", "sp.cu"]
+           "io_layers.cu", "sp.cu", "vae.cu"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",

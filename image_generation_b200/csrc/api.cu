@@ -142,6 +142,41 @@ Staging staging_plan(const h3dit_config *c) {
   return S;
 }
 
+// A VAE decoder context runs its layers through the block's machinery: the
+// same workspace plan with hidden = W, ffn = mlp, n_blocks = layers.
+bool vae_config_ok(const h3dit_vae_config *v) {
+  if (!v) return false;
+  if (v->width <= 0 || v->width % 64 || v->width > 8192) return false;
+  if (v->heads <= 0 || (v->head_dim != 96 && v->head_dim != 128)) return false;
+  if (v->mlp <= 0 || v->mlp % 64 || v->layers <= 0) return false;
+  if (v->tile <= 0 || v->channels < 1 || v->channels > 32 || v->max_tokens <= 0) return false;
+  return v->eps >= 0.f;
+}
+
+h3dit_config vae_internal(const h3dit_vae_config *v) {
+  h3dit_config c{};
+  c.hidden = v->width;
+  c.heads = v->heads;
+  c.head_dim = v->head_dim;
+  c.ffn = v->mlp < 768 ? 768 : v->mlp;  // the FFN buffer also holds the [n, 768] pixel rows
+  c.n_blocks = v->layers;
+  c.max_tokens = v->max_tokens;
+  c.rope_sections[0] = 16;
+  c.rope_sections[1] = c.rope_sections[2] = v->head_dim == 96 ? 16 : 24;
+  c.rope_theta = 10000.f;
+  c.norm_eps = v->eps;
+  c.t_scale = 1000.f;
+  c.precision = H3DIT_PRECISION_BF16;
+  return c;
+}
+
+// Workspace beyond the block plan: the position table [tile^2, W] and a
+// vector of W ones (the unit gate of the residual updates).
+size_t vae_extra_bytes(const h3dit_vae_config *v) {
+  const size_t W = v->width, T = v->tile;
+  return round_up(T * T * W * 4, kAlign) + round_up(W * 4, kAlign);
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -191,6 +226,12 @@ struct h3dit_ctx {
   bool own_copy = false;
   cudaEvent_t fork = nullptr, join = nullptr, ready[2] = {nullptr, nullptr},
               slot_free[2] = {nullptr, nullptr};
+  // a VAE decoder context (h3dit_vae_create): its layers and extra workspace
+  bool vae = false;
+  h3dit_vae_config vcfg{};
+  h3dit_vae_weights vw{};
+  std::vector<h3dit_vae_layer_weights> vlayers;
+  size_t vpos = 0, vones = 0;  // workspace offsets: position table, a vector of ones
 
   int *status() { return reinterpret_cast<int *>(ws + L.status); }
   float *resid() { return reinterpret_cast<float *>(ws + L.resid); }
@@ -329,7 +370,7 @@ h3dit_status encode_heads(h3dit_ctx *ctx, CUtensorMap *m, const void *base, int 
 
 h3dit_status run_linear(h3dit_ctx *ctx, int epi, const void *a, const void *w, int m, int n,
                         int k, void *out, long long ldo, const float *gate, const float *rope,
-                        cudaStream_t s) {
+                        cudaStream_t s, const float *bias = nullptr, int kind_override = -1) {
   if (epi < H3DIT_EPI_STORE || epi > H3DIT_EPI_GATED_RESIDUAL)
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "unknown epilogue %d", epi);
   if (m < 0 || n <= 0 || k <= 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "bad shape %d x %d x %d", m, n, k);
@@ -339,7 +380,10 @@ h3dit_status run_linear(h3dit_ctx *ctx, int epi, const void *a, const void *w, i
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "linear: NULL or misaligned pointer");
   if (epi == H3DIT_EPI_GATED_RESIDUAL && (!gate || !aligned16(gate)))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "gated residual needs a 16-byte aligned gate");
+  if (bias && (!aligned16(bias) || epi == H3DIT_EPI_QKV_ROPE))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "bias must be 16-byte aligned, and not with QKV + RoPE");
   GemmParams p{};
+  p.bias = bias;
   if (epi == H3DIT_EPI_QKV_ROPE) {
     const int I = ctx->inner(), dh = ctx->cfg.head_dim;
     const int *sec = ctx->cfg.rope_sections;
@@ -381,7 +425,8 @@ h3dit_status run_linear(h3dit_ctx *ctx, int epi, const void *a, const void *w, i
   p.status = ctx->status();
   const int tiles = p.tiles_m * p.tiles_n;
   const int grid = tiles < ctx->num_sms ? tiles : ctx->num_sms;
-  const int kind = epi == H3DIT_EPI_QKV_ROPE   ? H3DIT_KERNEL_QKV
+  const int kind = kind_override >= 0         ? kind_override
+                   : epi == H3DIT_EPI_QKV_ROPE ? H3DIT_KERNEL_QKV
                    : epi == H3DIT_EPI_GELU     ? H3DIT_KERNEL_FFN1
                    : k == ctx->inner()         ? H3DIT_KERNEL_OUT_PROJ
                    : epi == H3DIT_EPI_STORE    ? H3DIT_KERNEL_FFN1
@@ -485,9 +530,11 @@ h3dit_status run_linear_mx(h3dit_ctx *ctx, int epi, const void *a, const void *a
 
 h3dit_status run_attention(h3dit_ctx *ctx, const void *q, const void *k, const void *v, int ld,
                            void *o, int ldo, int n, cudaStream_t s, void *o_sf = nullptr,
-                           int heads = 0) {
+                           int heads = 0, int batch = 1) {
   if (heads == 0) heads = ctx->cfg.heads;
   if (n < 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "n < 0");
+  if (batch < 1 || static_cast<long long>(n) * batch > (1LL << 30))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "bad sequence batch");
   if (heads < 1 || heads > ctx->cfg.heads)
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "heads %d outside [1, %d]", heads, ctx->cfg.heads);
   if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
@@ -498,11 +545,13 @@ h3dit_status run_attention(h3dit_ctx *ctx, const void *q, const void *k, const v
   if (n == 0) return H3DIT_OK;
   CUtensorMap tq, tk, tv;
   h3dit_status st;
-  if ((st = encode_heads(ctx, &tq, q, n, heads, ctx->cfg.head_dim, ld, kAttnBQ))) return st;
-  if ((st = encode_heads(ctx, &tk, k, n, heads, ctx->cfg.head_dim, ld, kAttnBKV))) return st;
-  if ((st = encode_heads(ctx, &tv, v, n, heads, ctx->cfg.head_dim, ld, kAttnBKV))) return st;
+  const int rows = n * batch;
+  if ((st = encode_heads(ctx, &tq, q, rows, heads, ctx->cfg.head_dim, ld, kAttnBQ))) return st;
+  if ((st = encode_heads(ctx, &tk, k, rows, heads, ctx->cfg.head_dim, ld, kAttnBKV))) return st;
+  if ((st = encode_heads(ctx, &tv, v, rows, heads, ctx->cfg.head_dim, ld, kAttnBKV))) return st;
   AttnParams p{};
   p.n = n;
+  p.batch = batch;
   p.tiles_kv = (n + kAttnBKV - 1) / kAttnBKV;
   p.o = o;
   p.ldo = ldo;
@@ -721,6 +770,40 @@ h3dit_status run_blocks(h3dit_ctx *ctx, int l0, int l1, int n, cudaStream_t s,
   return ctx->cuda(cudaStreamWaitEvent(s, ctx->join, 0), "join wait");
 }
 
+h3dit_status run_layernorm(h3dit_ctx *ctx, const float *x, const float *g, const float *b,
+                           void *out, int n, cudaStream_t s) {
+  Launch L(ctx, H3DIT_KERNEL_RMSNORM, s);
+  return ctx->cuda(launch_layernorm(x, g, b, out, n, ctx->cfg.hidden, ctx->cfg.norm_eps,
+                                    ctx->num_sms, s),
+                   "layernorm launch");
+}
+
+// One decoder layer on the n tokens of `tiles` tiles in the fp32 residual.
+h3dit_status vae_layer(h3dit_ctx *ctx, const h3dit_vae_layer_weights &w, int n, int tiles,
+                       cudaStream_t s) {
+  const int W = ctx->cfg.hidden, I = ctx->inner(), M = ctx->vcfg.mlp;
+  const int per_tile = ctx->vcfg.tile * ctx->vcfg.tile;
+  const float *ones = reinterpret_cast<const float *>(ctx->ws + ctx->vones);
+  uint16_t *qkv = static_cast<uint16_t *>(ctx->qkv());
+  h3dit_status st = run_layernorm(ctx, ctx->resid(), w.ln1_g, w.ln1_b, ctx->xm(), n, s);
+  if (st) return st;
+  if ((st = run_linear(ctx, H3DIT_EPI_STORE, ctx->xm(), w.w_qkv, n, 3 * I, W, qkv, 3 * I, nullptr,
+                       nullptr, s, w.b_qkv, H3DIT_KERNEL_QKV)))
+    return st;
+  if ((st = run_attention(ctx, qkv, qkv + I, qkv + 2 * I, 3 * I, ctx->attn(), I, per_tile, s,
+                          nullptr, 0, tiles)))
+    return st;
+  if ((st = run_linear(ctx, H3DIT_EPI_GATED_RESIDUAL, ctx->attn(), w.w_o, n, W, I, ctx->resid(), W,
+                       ones, nullptr, s, w.b_o, H3DIT_KERNEL_OUT_PROJ)))
+    return st;
+  if ((st = run_layernorm(ctx, ctx->resid(), w.ln2_g, w.ln2_b, ctx->xm(), n, s))) return st;
+  if ((st = run_linear(ctx, H3DIT_EPI_GELU, ctx->xm(), w.w_1, n, M, W, ctx->u(), M, nullptr,
+                       nullptr, s, w.b_1, H3DIT_KERNEL_FFN1)))
+    return st;
+  return run_linear(ctx, H3DIT_EPI_GATED_RESIDUAL, ctx->u(), w.w_2, n, W, M, ctx->resid(), W, ones,
+                    nullptr, s, w.b_2, H3DIT_KERNEL_FFN2);
+}
+
 }  // namespace
 
 extern "C" {
@@ -929,6 +1012,7 @@ h3dit_status h3dit_sync_status(h3dit_ctx *ctx, void *cuda_stream) {
 
 h3dit_status h3dit_time_embed(h3dit_ctx *ctx, float t, float *c_out, void *cuda_stream) {
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (ctx->vae) return ctx->fail(H3DIT_ERR_UNSUPPORTED, "a decoder context runs h3dit_vae_decode");
   if (!c_out) return ctx->fail(H3DIT_ERR_INVALID_ARG, "c_out is NULL");
   const h3dit_time_weights &w = ctx->tw;
   Launch L(ctx, H3DIT_KERNEL_TIME_EMBED, static_cast<cudaStream_t>(cuda_stream), 2);
@@ -941,6 +1025,7 @@ h3dit_status h3dit_time_embed(h3dit_ctx *ctx, float t, float *c_out, void *cuda_
 h3dit_status h3dit_adaln_project(h3dit_ctx *ctx, const float *c, int32_t first, int32_t count,
                                  float *mod_out, void *cuda_stream) {
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (ctx->vae) return ctx->fail(H3DIT_ERR_UNSUPPORTED, "a decoder context runs h3dit_vae_decode");
   if (!c || !mod_out) return ctx->fail(H3DIT_ERR_INVALID_ARG, "NULL pointer");
   if (first < 0 || count < 0 || first + count > ctx->cfg.n_blocks)
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "block range [%d, %d) outside [0, %d)", first,
@@ -1109,6 +1194,7 @@ h3dit_status h3dit_block_forward(h3dit_ctx *ctx, int32_t block, float t, const f
                                  void *x_img, const h3dit_grid *grids, int32_t n_grids,
                                  void *x_txt, int32_t n_txt, void *cuda_stream) {
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (ctx->vae) return ctx->fail(H3DIT_ERR_UNSUPPORTED, "a decoder context runs h3dit_vae_decode");
   if (block < 0 || block >= ctx->cfg.n_blocks)
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "block %d outside [0, %d)", block, ctx->cfg.n_blocks);
   if (mod && !aligned16(mod)) return ctx->fail(H3DIT_ERR_INVALID_ARG, "mod is misaligned");
@@ -1130,6 +1216,7 @@ h3dit_status h3dit_block_forward(h3dit_ctx *ctx, int32_t block, float t, const f
 h3dit_status h3dit_step(h3dit_ctx *ctx, float t, void *x_img, const h3dit_grid *grids,
                         int32_t n_grids, void *x_txt, int32_t n_txt, void *cuda_stream) {
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (ctx->vae) return ctx->fail(H3DIT_ERR_UNSUPPORTED, "a decoder context runs h3dit_vae_decode");
   int n_img = 0;
   h3dit_status st = check_tokens(ctx, x_img, grids, n_grids, x_txt, n_txt, &n_img);
   if (st) return st;
@@ -1147,6 +1234,7 @@ h3dit_status h3dit_denoise(h3dit_ctx *ctx, const h3dit_io_weights *io, float *la
                            int32_t channels, int32_t lat_h, int32_t lat_w, const void *x_txt,
                            int32_t n_txt, int32_t n_steps, void *cuda_stream) {
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (ctx->vae) return ctx->fail(H3DIT_ERR_UNSUPPORTED, "a decoder context runs h3dit_vae_decode");
   if (!io || !io->w_in || !io->b_in || !io->w_mod || !io->b_mod || !io->w_out || !io->b_out ||
       !aligned16(io->w_in) || !aligned16(io->b_in))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "denoise: NULL or misaligned FP32 layer weights");
@@ -1200,6 +1288,138 @@ h3dit_status h3dit_denoise(h3dit_ctx *ctx, const h3dit_io_weights *io, float *la
       return st;
   }
   return H3DIT_OK;
+}
+
+size_t h3dit_vae_workspace_bytes(const h3dit_vae_config *cfg) {
+  if (!vae_config_ok(cfg)) return 0;
+  const h3dit_config ic = vae_internal(cfg);
+  return plan(&ic).total + vae_extra_bytes(cfg);
+}
+
+h3dit_status h3dit_vae_create(const h3dit_vae_config *cfg, const h3dit_vae_weights *w,
+                              void *workspace, size_t ws_bytes, void *cuda_stream,
+                              h3dit_ctx **out) {
+  if (!out) return H3DIT_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!vae_config_ok(cfg) || !w || !w->layers) return H3DIT_ERR_INVALID_ARG;
+  const void *need[] = {w->w_in, w->b_in, w->lnf_g, w->lnf_b, w->w_out, w->b_out};
+  for (const void *p : need)
+    if (!p || !aligned16(p)) return H3DIT_ERR_INVALID_ARG;
+  for (int l = 0; l < cfg->layers; ++l) {
+    const h3dit_vae_layer_weights &v = w->layers[l];
+    const void *lp[] = {v.ln1_g, v.ln1_b, v.w_qkv, v.b_qkv, v.w_o, v.b_o,
+                        v.ln2_g, v.ln2_b, v.w_1, v.b_1, v.w_2, v.b_2};
+    for (const void *p : lp)
+      if (!p || !aligned16(p)) return H3DIT_ERR_INVALID_ARG;
+  }
+  const h3dit_config ic = vae_internal(cfg);
+  const Layout L = plan(&ic);
+  const size_t total = L.total + vae_extra_bytes(cfg);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) || ws_bytes < total)
+    return H3DIT_ERR_WORKSPACE;
+  h3dit_ctx *ctx = new (std::nothrow) h3dit_ctx();
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  ctx->cfg = ic;
+  ctx->vae = true;
+  ctx->vcfg = *cfg;
+  ctx->vlayers.assign(w->layers, w->layers + cfg->layers);
+  ctx->vw = *w;
+  ctx->vw.layers = ctx->vlayers.data();
+  ctx->ws = static_cast<uint8_t *>(workspace);
+  ctx->ws_bytes = ws_bytes;
+  ctx->L = L;
+  ctx->vpos = L.total;
+  ctx->vones = L.total + round_up(static_cast<size_t>(cfg->tile) * cfg->tile * cfg->width * 4, kAlign);
+  ctx->streamed.assign(cfg->layers, 0);
+  int dev = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    delete ctx;
+    return H3DIT_ERR_CUDA;
+  }
+  std::vector<float> ones(cfg->width, 1.0f);
+  cudaError_t e = cudaMemsetAsync(ctx->status(), 0, sizeof(int), s);
+  if (e == cudaSuccess)
+    e = launch_vae_pos_table(cfg->tile, cfg->width, reinterpret_cast<float *>(ctx->ws + ctx->vpos),
+                             ctx->num_sms, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(ctx->ws + ctx->vones, ones.data(), ones.size() * sizeof(float),
+                        cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);  // the host vector dies with this call
+  if (e != cudaSuccess) {
+    delete ctx;
+    return H3DIT_ERR_CUDA;
+  }
+  *out = ctx;
+  return H3DIT_OK;
+}
+
+h3dit_status h3dit_vae_decode(h3dit_ctx *ctx, const float *latent, int32_t lat_h, int32_t lat_w,
+                              float *image, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (!ctx->vae) return ctx->fail(H3DIT_ERR_UNSUPPORTED, "not a decoder context (h3dit_vae_create)");
+  if (!latent || !image || !aligned16(latent) || !aligned16(image))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "decode: NULL or misaligned latent or image");
+  const int T = ctx->vcfg.tile;
+  if (lat_h < 1 || lat_w < 1) return ctx->fail(H3DIT_ERR_INVALID_ARG, "empty latent");
+  if (lat_h % T || lat_w % T)
+    return ctx->fail(H3DIT_ERR_UNSUPPORTED, "latent sides %d x %d are not multiples of the tile %d",
+                     lat_h, lat_w, T);
+  const long long n = static_cast<long long>(lat_h) * lat_w;
+  if (n > ctx->cfg.max_tokens)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "%lld tokens exceed max_tokens=%d", n, ctx->cfg.max_tokens);
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  const int W = ctx->cfg.hidden, tiles = static_cast<int>(n / (static_cast<long long>(T) * T));
+  h3dit_status st;
+  {
+    Launch L(ctx, H3DIT_KERNEL_IO, s);
+    if ((st = ctx->cuda(launch_vae_embed(latent, ctx->vcfg.channels, lat_h, lat_w, T, ctx->vw.w_in,
+                                         ctx->vw.b_in,
+                                         reinterpret_cast<const float *>(ctx->ws + ctx->vpos), W,
+                                         ctx->resid(), s),
+                        "decoder embedding launch")))
+      return st;
+  }
+  for (int l = 0; l < ctx->vcfg.layers; ++l)
+    if ((st = vae_layer(ctx, ctx->vlayers[l], static_cast<int>(n), tiles, s))) return st;
+  if ((st = run_layernorm(ctx, ctx->resid(), ctx->vw.lnf_g, ctx->vw.lnf_b, ctx->xm(),
+                          static_cast<int>(n), s)))
+    return st;
+  if ((st = run_linear(ctx, H3DIT_EPI_STORE, ctx->xm(), ctx->vw.w_out, static_cast<int>(n), 768, W,
+                       ctx->u(), 768, nullptr, nullptr, s, ctx->vw.b_out, H3DIT_KERNEL_IO)))
+    return st;
+  Launch L(ctx, H3DIT_KERNEL_IO, s);
+  return ctx->cuda(launch_vae_pixels(ctx->u(), lat_h, lat_w, T, image, ctx->num_sms, s),
+                   "decoder pixels launch");
+}
+
+h3dit_status h3dit_layernorm(h3dit_ctx *ctx, const float *x, const float *gain, const float *bias,
+                             void *out, int32_t n, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (n < 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "n < 0");
+  if (!x || !gain || !bias || !out || !aligned16(x) || !aligned16(gain) || !aligned16(bias) ||
+      !aligned16(out))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "NULL or misaligned pointer");
+  if (n == 0) return H3DIT_OK;
+  return run_layernorm(ctx, x, gain, bias, out, n, static_cast<cudaStream_t>(cuda_stream));
+}
+
+h3dit_status h3dit_linear_bias(h3dit_ctx *ctx, int32_t epilogue, const void *a, const void *w,
+                               const float *bias, int32_t m, int32_t n, int32_t k, void *out,
+                               const float *gate, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (!bias) return ctx->fail(H3DIT_ERR_INVALID_ARG, "bias is NULL");
+  return run_linear(ctx, epilogue, a, w, m, n, k, out, n, gate, nullptr,
+                    static_cast<cudaStream_t>(cuda_stream), bias);
+}
+
+h3dit_status h3dit_attention_batched(h3dit_ctx *ctx, const void *q, const void *k, const void *v,
+                                     int32_t ld_qkv, void *o, int32_t ld_o, int32_t n,
+                                     int32_t batch, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  return run_attention(ctx, q, k, v, ld_qkv, o, ld_o, n, static_cast<cudaStream_t>(cuda_stream),
+                       nullptr, 0, batch);
 }
 
 size_t h3dit_mx_scale_bytes(int32_t rows, int32_t k) {

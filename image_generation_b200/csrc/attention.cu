@@ -148,6 +148,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int lane = threadIdx.x & 31;
   const int head = blockIdx.y;
   const int q0 = blockIdx.x * 2 * BQ;
+  // sequence blockIdx.z of a batch of equal-length sequences stored one after
+  // another (rows z n .. z n + n - 1); query rows past n are computed but not
+  // stored, keys past n are masked below
+  const int seq0 = blockIdx.z * p.n;
   const int nkv = p.tiles_kv;
 
   if (threadIdx.x == 0) {
@@ -185,7 +189,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive_expect_tx(Q_FULL, 2 * DCH * QBOX);
       for (int t = 0; t < 2; ++t)
         for (int c = 0; c < DCH; ++c)
-          tma_load_3d(sQ + t * Q_BYTES + c * QBOX, &tq, 64 * c, head, q0 + t * BQ, Q_FULL);
+          tma_load_3d(sQ + t * Q_BYTES + c * QBOX, &tq, 64 * c, head, seq0 + q0 + t * BQ, Q_FULL);
       int issued = 0;
       for (int j = 0; j < nkv; ++j) {
         const int st = j % NS;
@@ -194,8 +198,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t k_dst = sKV + st * STAGE_BYTES;
         const uint32_t v_dst = k_dst + KV_BYTES;
         for (int c = 0; c < DCH; ++c) {
-          tma_load_3d(k_dst + c * KBOX, &tk, 64 * c, head, j * BKV, KV_FULL(st));
-          tma_load_3d(v_dst + c * KBOX, &tv, 64 * c, head, j * BKV, KV_FULL(st));
+          tma_load_3d(k_dst + c * KBOX, &tk, 64 * c, head, seq0 + j * BKV, KV_FULL(st));
+          tma_load_3d(v_dst + c * KBOX, &tv, 64 * c, head, seq0 + j * BKV, KV_FULL(st));
         }
         issued = j + 1;
       }
@@ -324,8 +328,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const float inv_l = 1.f / l;
-      const int qrow = q0 + t * BQ + row;
-      uint16_t *dst = static_cast<uint16_t *>(p.o) + static_cast<size_t>(qrow) * p.ldo + head * DH;
+      const int qrow = q0 + t * BQ + row;  // within the sequence
+      const size_t grow = static_cast<size_t>(seq0) + qrow;
+      uint16_t *dst = static_cast<uint16_t *>(p.o) + grow * p.ldo + head * DH;
 #pragma unroll
       for (int c = 0; c < DH / 32; ++c) {
         uint32_t r[32];
@@ -337,11 +342,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * inv_l;
             uint32_t q[8];
             const uint32_t sb = mx_quant32(v, q);
-            uint8_t *d8 = static_cast<uint8_t *>(p.o) + static_cast<size_t>(qrow) * p.ldo +
+            uint8_t *d8 = static_cast<uint8_t *>(p.o) + grow * p.ldo +
                           head * DH + 32 * c;
             st_global_v4(d8, q[0], q[1], q[2], q[3]);
             st_global_v4(d8 + 16, q[4], q[5], q[6], q[7]);
-            p.o_sf[mx_sf_offset(qrow, (head * DH) / 32 + c, static_cast<int>(p.ldo / 128))] =
+            p.o_sf[mx_sf_offset(static_cast<int>(grow), (head * DH) / 32 + c,
+                                static_cast<int>(p.ldo / 128))] =
                 static_cast<uint8_t>(sb);
           }
           continue;
@@ -378,7 +384,7 @@ cudaError_t launch_dh(const CUtensorMap &q, const CUtensorMap &k, const CUtensor
   static PerDevice smem_attr;
   cudaError_t e = set_smem_once(smem_attr, attn_fwd_tcgen05<DH, OUT_MX>, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.n + 2 * BQ - 1) / (2 * BQ), heads);
+  dim3 grid((p.n + 2 * BQ - 1) / (2 * BQ), heads, p.batch);
   attn_fwd_tcgen05<DH, OUT_MX><<<grid, THREADS, SMEM_BYTES, s>>>(q, k, v, p);
   return cudaGetLastError();
 }

@@ -2,7 +2,8 @@
 // owns one output row of the tile (its TMEM lane) and walks the tile's columns
 // in 32-column chunks (48 for a 24-pair rotary section), applying the fused
 // step: plain bf16 store, RoPE on Q and K, GELU (bf16 or MXFP8 out), or the
-// AdaLN-gated residual update of the fp32 stream.
+// AdaLN-gated residual update of the fp32 stream; with a bias vector (the VAE
+// decoder's linears) the bias is added to the product first.
 #pragma once
 
 #include <cuda_fp8.h>
@@ -106,6 +107,17 @@ __device__ __forceinline__ void plain_chunk(const GemmParams &p, uint32_t taddr,
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  if (p.bias) {
+    const float4 *b = reinterpret_cast<const float4 *>(p.bias + col);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 bb = __ldg(b + q);
+      v[4 * q + 0] += bb.x;
+      v[4 * q + 1] += bb.y;
+      v[4 * q + 2] += bb.z;
+      v[4 * q + 3] += bb.w;
+    }
+  }
   if constexpr (EPI == kEpiGatedResidual) {
     float4 *x = reinterpret_cast<float4 *>(static_cast<float *>(p.out) +
                                            static_cast<size_t>(row) * p.ldo + col);

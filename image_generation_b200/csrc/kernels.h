@@ -84,6 +84,7 @@ struct GemmParams {
   void *out;
   long long ldo;          // elements
   const float *gate;      // gated residual: [n]
+  const float *bias;      // optional [n], added to the product before the epilogue step
   const float *rope;      // QKV: [m][head_dim/2][2]
   int head_dim;           // QKV
   int rope_cols;          // QKV: RoPE on columns < rope_cols (Q and K)
@@ -96,7 +97,8 @@ struct GemmParams {
 };
 
 struct AttnParams {
-  int n;                  // tokens
+  int n;                  // tokens of one sequence (blockIdx.z picks the sequence)
+  int batch;              // sequences, stored one after another (rows z n .. z n + n - 1)
   int tiles_kv;
   void *o;
   long long ldo;          // elements
@@ -161,6 +163,15 @@ cudaError_t launch_sp_pack_qkv(const void *qkv, int n, int ranks, int cw, void *
                                cudaStream_t s);
 cudaError_t launch_sp_unpack_o(const void *recv, int n, int ranks, int cw, void *o, int num_sms,
                                cudaStream_t s);
+// The VAE decoder's own steps (vae.cu).
+cudaError_t launch_layernorm(const float *x, const float *gain, const float *bias, void *out,
+                             int n, int d, float eps, int num_sms, cudaStream_t s);
+cudaError_t launch_vae_pos_table(int T, int W, float *table, int num_sms, cudaStream_t s);
+cudaError_t launch_vae_embed(const float *z, int C, int Hl, int Wl, int T, const float *w_in,
+                             const float *b_in, const float *table, int W, float *out,
+                             cudaStream_t s);
+cudaError_t launch_vae_pixels(const void *tokens, int Hl, int Wl, int T, float *img, int num_sms,
+                              cudaStream_t s);
 cudaError_t launch_mx_tile_sf(const uint8_t *sf, int n, int k, uint8_t *tiled, cudaStream_t s);
 // bf16 [rows, k] (row stride ld elements) -> E4M3 [rows, k] + scales.
 cudaError_t launch_mx_quantize(const void *src, long long ld, int rows, int k, uint8_t *dst,

@@ -66,6 +66,23 @@ class h3dit_io_weights(C.Structure):
                 ("b_mod", C.c_void_p), ("w_out", C.c_void_p), ("b_out", C.c_void_p)]
 
 
+class h3dit_vae_config(C.Structure):
+    _fields_ = [("width", C.c_int32), ("heads", C.c_int32), ("head_dim", C.c_int32),
+                ("mlp", C.c_int32), ("layers", C.c_int32), ("tile", C.c_int32),
+                ("channels", C.c_int32), ("max_tokens", C.c_int32), ("eps", C.c_float)]
+
+
+class h3dit_vae_layer_weights(C.Structure):
+    _fields_ = [(k, C.c_void_p) for k in ("ln1_g", "ln1_b", "w_qkv", "b_qkv", "w_o", "b_o",
+                                           "ln2_g", "ln2_b", "w_1", "b_1", "w_2", "b_2")]
+
+
+class h3dit_vae_weights(C.Structure):
+    _fields_ = [("w_in", C.c_void_p), ("b_in", C.c_void_p),
+                ("layers", C.POINTER(h3dit_vae_layer_weights)), ("lnf_g", C.c_void_p),
+                ("lnf_b", C.c_void_p), ("w_out", C.c_void_p), ("b_out", C.c_void_p)]
+
+
 class h3dit_grid(C.Structure):
     _fields_ = [("frame", C.c_int32), ("height", C.c_int32), ("width", C.c_int32)]
 
@@ -113,6 +130,13 @@ def _load() -> C.CDLL:
         "h3dit_attention_heads": (i32, [p, i32, p, p, p, i32, p, i32, i32, p]),
         "h3dit_sp_pack_qkv": (i32, [p, p, i32, i32, p, p]),
         "h3dit_sp_unpack_o": (i32, [p, p, i32, i32, p, p]),
+        "h3dit_vae_workspace_bytes": (sz, [C.POINTER(h3dit_vae_config)]),
+        "h3dit_vae_create": (i32, [C.POINTER(h3dit_vae_config), C.POINTER(h3dit_vae_weights), p,
+                                   sz, p, C.POINTER(p)]),
+        "h3dit_vae_decode": (i32, [p, p, i32, i32, p, p]),
+        "h3dit_layernorm": (i32, [p, p, p, p, p, i32, p]),
+        "h3dit_linear_bias": (i32, [p, i32, p, p, p, i32, i32, i32, p, p, p]),
+        "h3dit_attention_batched": (i32, [p, p, p, p, i32, p, i32, i32, i32, p]),
         "h3dit_staging_bytes": (sz, [C.POINTER(h3dit_config)]),
         "h3dit_attach_staging": (i32, [p, p, sz, p]),
         "h3dit_streamed_blocks": (i32, [p]),
@@ -244,6 +268,22 @@ class Context:
                               ws_bytes, _stream(stream), C.byref(handle))
         check(None, st)
         self.handle = handle
+
+    def layernorm(self, x, gain, bias, out, stream=None) -> None:
+        self._check(lib.h3dit_layernorm(self.handle, _ptr(x), _ptr(gain), _ptr(bias), _ptr(out),
+                                        x.shape[0], _stream(stream)))
+
+    def linear_bias(self, epilogue: int, a, w, bias, out, gate=None, stream=None) -> None:
+        m, k = a.shape
+        n = w.shape[0]
+        self._check(lib.h3dit_linear_bias(self.handle, epilogue, _ptr(a), _ptr(w), _ptr(bias), m,
+                                          n, k, _ptr(out), _ptr(gate), _stream(stream)))
+
+    def attention_batched(self, q, k, v, ld_qkv: int, o, ld_o: int, n: int, batch: int,
+                          stream=None) -> None:
+        self._check(lib.h3dit_attention_batched(self.handle, _ptr(q, False), _ptr(k, False),
+                                                _ptr(v, False), ld_qkv, _ptr(o, False), ld_o, n,
+                                                batch, _stream(stream)))
 
     def attach_staging(self, staging=None, copy_stream=None) -> None:
         """Lend the context device staging memory for blocks whose weights are
@@ -410,3 +450,46 @@ class Context:
         n_txt = 0 if x_txt is None else x_txt.shape[0]
         self._check(lib.h3dit_step(self.handle, t, _ptr(x_img), g, len(grids), _ptr(x_txt),
                                    n_txt, _stream(stream)))
+
+
+def make_vae_config(width=1280, heads=10, head_dim=128, mlp=5120, layers=24, tile=32,
+                    channels=24, max_tokens=65536, eps=1e-6) -> h3dit_vae_config:
+    return h3dit_vae_config(width, heads, head_dim, mlp, layers, tile, channels, max_tokens, eps)
+
+
+class VaeDecoder(Context):
+    """A decoder context (h3dit_vae_create) holding the torch tensors it
+    borrows. weights: w_in, b_in, lnf_g, lnf_b, w_out, b_out and "layers", a
+    list of dicts with ln1_g, ln1_b, w_qkv, b_qkv, w_o, b_o, ln2_g, ln2_b, w_1,
+    b_1, w_2, b_2 (matrices bf16, vectors fp32, all on the device)."""
+
+    def __init__(self, cfg: h3dit_vae_config, weights: dict, stream=None, workspace=None):
+        import torch
+
+        self.cfg = cfg
+        self._keep = [weights]
+        ws_bytes = lib.h3dit_vae_workspace_bytes(C.byref(cfg))
+        if ws_bytes == 0:
+            raise H3DitError(H3DIT_ERR_INVALID_ARG, "invalid decoder config")
+        if workspace is None:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        self.workspace = workspace
+        names = [f[0] for f in h3dit_vae_layer_weights._fields_]
+        layers = (h3dit_vae_layer_weights * len(weights["layers"]))()
+        for i, lw in enumerate(weights["layers"]):
+            layers[i] = h3dit_vae_layer_weights(*[_ptr(lw[k]) for k in names])
+        self._layers = layers
+        vw = h3dit_vae_weights(_ptr(weights["w_in"]), _ptr(weights["b_in"]), layers,
+                               _ptr(weights["lnf_g"]), _ptr(weights["lnf_b"]),
+                               _ptr(weights["w_out"]), _ptr(weights["b_out"]))
+        handle = C.c_void_p()
+        st = lib.h3dit_vae_create(C.byref(cfg), C.byref(vw), _ptr(workspace), ws_bytes,
+                                  _stream(stream), C.byref(handle))
+        check(None, st)
+        self.handle = handle
+
+    def decode(self, latent, image, stream=None) -> None:
+        """latent fp32 [C, Hl, Wl] -> image fp32 [3, 16 Hl, 16 Wl]."""
+        _, h, w = latent.shape
+        self._check(lib.h3dit_vae_decode(self.handle, _ptr(latent), h, w, _ptr(image),
+                                         _stream(stream)))

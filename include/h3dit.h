@@ -394,6 +394,101 @@ h3dit_status h3dit_denoise(h3dit_ctx *ctx, const h3dit_io_weights *io, float *la
                            int32_t channels, int32_t lat_h, int32_t lat_w, const void *x_txt,
                            int32_t n_txt, int32_t n_steps, void *cuda_stream);
 
+/* ---- The image VAE's ViT decoder (shape level) -------------------------
+ * MiniMax-H3-Image model card, "Model Architecture": the image VAE has a CNN
+ * encoder and a 2D ViT decoder with 24 layers, 16x spatial downsampling and
+ * 24 latent channels. "H3-Image Day-0 Support: 4K in 0.87s with Vera Rubin",
+ * "Faster Decoding": the VAE decodes independent image tiles. The pages give
+ * no more, so the decoder is a plain reading of those words, run on random
+ * weights for its shape and cost:
+ *   - one token per latent pixel: Linear(C -> W) + bias, plus a fixed 2-D
+ *     sin-cos position table over the position inside the tile (first W/2
+ *     channels the row r, last W/2 the column c, each [sin(p w_k) | cos(p w_k)]
+ *     for k < W/4 with w_k = 10000^(-k/(W/4)));
+ *   - `layers` pre-norm ViT layers: x += (attention over the tile's tokens of
+ *     LN1(x) W_qkv^T + b_qkv) W_o^T + b_o; x += GELU(LN2(x) W_1^T + b_1) W_2^T
+ *     + b_2; LayerNorm with gain and bias; attention unmasked, scale
+ *     1/sqrt(head_dim), no rotary embedding;
+ *   - a final LayerNorm, Linear(W -> 3*16*16) + bias, and each token's 768
+ *     outputs as its 16 x 16 RGB pixel block (feature ch*256 + 16i + j at
+ *     pixel (16r + i, 16c + j) of channel ch);
+ *   - the latent cut into non-overlapping tile x tile pieces decoded
+ *     independently (all tiles of a call at once: the row-wise steps over all
+ *     tokens, the attention batched over tiles).
+ * Linears run on bf16 operands with fp32 accumulation (the pages report a
+ * BF16 decode control; the checkpoint is FP32); the residual stream is fp32. */
+
+typedef struct h3dit_vae_config {
+  int32_t width;      /* W, multiple of 64 (1280)                                 */
+  int32_t heads;      /* attention heads (10)                                     */
+  int32_t head_dim;   /* 96 or 128 (128)                                          */
+  int32_t mlp;        /* MLP width, multiple of 64 (5120)                         */
+  int32_t layers;     /* ViT layers (24)                                          */
+  int32_t tile;       /* latent pixels per tile side (32 = 512 image pixels)      */
+  int32_t channels;   /* latent channels, 1 .. 32 (24)                            */
+  int32_t max_tokens; /* largest latent Hl*Wl a decode will pass                  */
+  float eps;          /* LayerNorm epsilon (1e-6)                                 */
+} h3dit_vae_config;
+
+/* One decoder layer: bf16 matrices in the nn.Linear layout, fp32 vectors,
+ * all device memory borrowed for the context's life. */
+typedef struct h3dit_vae_layer_weights {
+  const float *ln1_g, *ln1_b; /* [W]                                                  */
+  const void *w_qkv;          /* [3 H d, W]; rows [Q heads | K heads | V heads]       */
+  const float *b_qkv;         /* [3 H d]                                              */
+  const void *w_o;            /* [W, H d]                                             */
+  const float *b_o;           /* [W]                                                  */
+  const float *ln2_g, *ln2_b; /* [W]                                                  */
+  const void *w_1;            /* [mlp, W]                                             */
+  const float *b_1;           /* [mlp]                                                */
+  const void *w_2;            /* [W, mlp]                                             */
+  const float *b_2;           /* [W]                                                  */
+} h3dit_vae_layer_weights;
+
+typedef struct h3dit_vae_weights {
+  const float *w_in, *b_in;              /* fp32 [W, C], [W]                          */
+  const h3dit_vae_layer_weights *layers; /* host array of cfg->layers                 */
+  const float *lnf_g, *lnf_b;            /* [W]                                       */
+  const void *w_out;                     /* bf16 [768, W]                             */
+  const float *b_out;                    /* [768]                                     */
+} h3dit_vae_weights;
+
+/* Device workspace a decoder context needs, or 0 if `cfg` is invalid. */
+size_t h3dit_vae_workspace_bytes(const h3dit_vae_config *cfg);
+
+/* A decoder context (used with h3dit_vae_decode, the stage entry points
+ * below, h3dit_sync_status, the profile hooks and h3dit_destroy; the DiT
+ * calls refuse it). Workspace as in h3dit_create. Writes the position table
+ * into the workspace on `cuda_stream` and synchronises it once. */
+h3dit_status h3dit_vae_create(const h3dit_vae_config *cfg, const h3dit_vae_weights *w,
+                              void *workspace, size_t ws_bytes, void *cuda_stream,
+                              h3dit_ctx **out);
+
+/* latent device fp32 [C, Hl, Wl] -> image device fp32 [3, 16 Hl, 16 Wl].
+ * Hl and Wl must be multiples of cfg->tile (H3DIT_ERR_UNSUPPORTED otherwise)
+ * and Hl*Wl <= max_tokens. */
+h3dit_status h3dit_vae_decode(h3dit_ctx *ctx, const float *latent, int32_t lat_h, int32_t lat_w,
+                              float *image, void *cuda_stream);
+
+/* LayerNorm with gain and bias: x device fp32 [n, width] -> out device bf16
+ * [n, width] (width = the context's hidden, or W of a decoder context). */
+h3dit_status h3dit_layernorm(h3dit_ctx *ctx, const float *x, const float *gain, const float *bias,
+                             void *out, int32_t n, void *cuda_stream);
+
+/* h3dit_linear with a bias b (device fp32 [n]) added to the product before the
+ * epilogue step: STORE and GELU write bf16 (a w^T + b), GATED_RESIDUAL adds
+ * gate * (a w^T + b) to the fp32 out; QKV_ROPE is not offered with a bias. */
+h3dit_status h3dit_linear_bias(h3dit_ctx *ctx, int32_t epilogue, const void *a, const void *w,
+                               const float *bias, int32_t m, int32_t n, int32_t k, void *out,
+                               const float *gate, void *cuda_stream);
+
+/* a5 over `batch` independent sequences of n tokens stored one after another
+ * (rows z*n .. z*n + n - 1 of q, k, v and o): as h3dit_attention_heads with
+ * heads = cfg heads, each sequence attending only to itself. */
+h3dit_status h3dit_attention_batched(h3dit_ctx *ctx, const void *q, const void *k, const void *v,
+                                     int32_t ld_qkv, void *o, int32_t ld_o, int32_t n,
+                                     int32_t batch, void *cuda_stream);
+
 /* ---- Timestep condition without any device allocation ----------------- */
 
 /* Largest `hidden` h3dit_time_embed_static accepts. */
