@@ -723,6 +723,69 @@ def vae_timing(reps: int = 5) -> dict:
     return out
 
 
+def denoise_timing(ctx, x_txt, rank, world, barrier, dist, stream, reps: int = 2) -> dict:
+    """The whole 6-step sampling loop in one call (h3dit_denoise) on the 4096^2
+    latent [24, 256, 256]: on the device, and end to end with the noise and
+    the text states copied in from pinned host memory and the denoised latent
+    copied back, all inside the timed region."""
+    import torch
+
+    g = torch.Generator(device="cuda")
+    g.manual_seed(2000 + rank)
+    k4 = 4 * C_LAT
+    rnd = lambda *s: torch.randn(*s, device="cuda", generator=g) * 0.02
+    io = {"w_in": rnd(D, k4), "b_in": torch.zeros(D, device="cuda"), "w_mod": rnd(2 * D, D),
+          "b_mod": torch.zeros(2 * D, device="cuda"), "w_out": rnd(k4, D),
+          "b_out": torch.zeros(k4, device="cuda")}
+    shape = (C_LAT, 2 * GRID, 2 * GRID)
+    noise = torch.randn(*shape, device="cuda", generator=g)
+    lat = torch.empty_like(noise)
+    h_noise = torch.empty(shape, pin_memory=True)
+    h_noise.copy_(noise)
+    h_txt = torch.empty(x_txt.shape, dtype=x_txt.dtype, pin_memory=True)
+    h_txt.copy_(x_txt)
+    h_out = torch.empty(shape, pin_memory=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    lat.copy_(noise)
+    ctx.denoise(io, lat, x_txt, 6)  # warm-up
+    barrier()
+    e0.record(stream)
+    for _ in range(reps):
+        lat.copy_(noise)
+        ctx.denoise(io, lat, x_txt, 6)
+    e1.record(stream)
+    barrier()
+    d_ms = slowest_rank(e0.elapsed_time(e1), dist) / reps
+    e0.record(stream)
+    for _ in range(reps):
+        lat.copy_(h_noise, non_blocking=True)
+        x_txt.copy_(h_txt, non_blocking=True)
+        ctx.denoise(io, lat, x_txt, 6)
+        h_out.copy_(lat, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    de_ms = slowest_rank(e0.elapsed_time(e1), dist) / reps
+    if ctx.sync_status() != 0:
+        raise RuntimeError("denoise failed")
+    if not bool(torch.isfinite(h_out).all()):
+        raise RuntimeError("denoise produced non-finite values")
+    in_bytes = h_noise.numel() * 4 + h_txt.numel() * h_txt.element_size()
+    return {"ms": round(d_ms / world, 1), "steps": 6, "latent": list(shape),
+            "e2e": {"value": round(de_ms / world, 1), "unit": "ms",
+                    "h2d_bytes_per_run": in_bytes, "d2h_bytes_per_run": h_out.numel() * 4}}
+
+
+def optional_leg(name: str, fn):
+    """Run one of the extra measurements; a failure there is reported in its
+    field instead of costing the whole line (the step's own timing is not
+    guarded)."""
+    try:
+        return fn()
+    except Exception as e:  # noqa: BLE001 - reported, not hidden
+        print(f"bench: {name} failed: {e}", file=sys.stderr, flush=True)
+        return {"error": f"{type(e).__name__}: {str(e).splitlines()[0][:200]}"}
+
+
 def block_flops(n: int, d) -> float:
     I = d.heads * d.head_dim
     return 8.0 * n * d.hidden * I + 4.0 * n * d.hidden * d.ffn + 4.0 * n * n * I
@@ -834,67 +897,22 @@ def run_h3dit(args):
         if ctx.sync_status() != 0:
             raise RuntimeError("end-to-end steps failed")
 
-    # the whole 6-step sampling loop in one call (h3dit_denoise) on the 4096^2
-    # latent [24, 256, 256]: on the device, and end to end with the noise and
-    # the text states copied in from pinned host memory and the denoised
-    # latent copied back, all inside the timed region
     denoise = None
     if not args.no_denoise:
-        g = torch.Generator(device="cuda")
-        g.manual_seed(2000 + rank)
-        k4 = 4 * C_LAT
-        rnd = lambda *s: torch.randn(*s, device="cuda", generator=g) * 0.02
-        io = {"w_in": rnd(D, k4), "b_in": torch.zeros(D, device="cuda"), "w_mod": rnd(2 * D, D),
-              "b_mod": torch.zeros(2 * D, device="cuda"), "w_out": rnd(k4, D),
-              "b_out": torch.zeros(k4, device="cuda")}
-        shape = (C_LAT, 2 * GRID, 2 * GRID)
-        noise = torch.randn(*shape, device="cuda", generator=g)
-        lat = torch.empty_like(noise)
-        h_noise = torch.empty(shape, pin_memory=True)
-        h_noise.copy_(noise)
-        h_txt = torch.empty(x_txt.shape, dtype=x_txt.dtype, pin_memory=True)
-        h_txt.copy_(x_txt)
-        h_out = torch.empty(shape, pin_memory=True)
-        lat.copy_(noise)
-        ctx.denoise(io, lat, x_txt, 6)  # warm-up
-        barrier()
-        reps = 2
-        e0.record(stream)
-        for _ in range(reps):
-            lat.copy_(noise)
-            ctx.denoise(io, lat, x_txt, 6)
-        e1.record(stream)
-        barrier()
-        d_ms = slowest_rank(e0.elapsed_time(e1), dist) / reps
-        e0.record(stream)
-        for _ in range(reps):
-            lat.copy_(h_noise, non_blocking=True)
-            x_txt.copy_(h_txt, non_blocking=True)
-            ctx.denoise(io, lat, x_txt, 6)
-            h_out.copy_(lat, non_blocking=True)
-        e1.record(stream)
-        barrier()
-        de_ms = slowest_rank(e0.elapsed_time(e1), dist) / reps
-        if ctx.sync_status() != 0:
-            raise RuntimeError("denoise failed")
-        if not bool(torch.isfinite(h_out).all()):
-            raise RuntimeError("denoise produced non-finite values")
-        in_bytes = h_noise.numel() * 4 + h_txt.numel() * h_txt.element_size()
-        denoise = {"ms": round(d_ms / world, 1), "steps": 6, "latent": list(shape),
-                   "e2e": {"value": round(de_ms / world, 1), "unit": "ms",
-                           "h2d_bytes_per_run": in_bytes,
-                           "d2h_bytes_per_run": h_out.numel() * 4}}
-        del io, noise, lat
+        denoise = optional_leg("denoise", lambda: denoise_timing(ctx, x_txt, rank, world, barrier,
+                                                                 dist, stream))
 
     vae = None
     if world == 1 and not args.no_vae:
-        vae = vae_timing()
+        vae = optional_leg("vae", vae_timing)
 
     streaming = None
     if world == 1 and not args.no_streaming:
-        streaming = streaming_timings(tw, blocks, x_txt, x_img, grids, dh)
-        streaming["resident_50"] = {"ms_per_step": round(ms_step, 1), "streamed_blocks": 0,
-                                    "h2d_bytes_per_step": 0}
+        streaming = optional_leg("streaming", lambda: streaming_timings(tw, blocks, x_txt, x_img,
+                                                                        grids, dh))
+        if "error" not in streaming:
+            streaming["resident_50"] = {"ms_per_step": round(ms_step, 1), "streamed_blocks": 0,
+                                        "h2d_bytes_per_step": 0}
 
     line = None
     if rank == 0:
@@ -964,43 +982,53 @@ def run_h3dit(args):
             "gemm": round(line.get("gemm_tflops", 0.0) / NOMINAL_BF16_TFLOPS, 4),
             "attention": round((line.get("attention_tflops") or 0.0) / NOMINAL_BF16_TFLOPS, 4)}
         if world == 1 and not args.no_configs:
-            line["ms_per_block"] = block_timings(96)
-            line["ms_per_block"].update(block_timings(128))
+            def per_shape():
+                out = block_timings(96)
+                out.update(block_timings(128))
+                return out
+            line["ms_per_block"] = optional_leg("ms_per_block", per_shape)
         if world == 1 and not args.no_cpu_baseline:
-            v, desc, threads, secs = oracle_sample(dh)
-            line["cpu_baseline"] = {"value": round(v, 1), "unit": "ms", "cores": threads,
-                                    "kind": "oracle", "estimated": True, "sample": desc,
-                                    "sample_cpu_seconds": round(secs, 1)}
-            b_ms, b_desc, b_threads = oracle_block_2k(dh)
-            line["cpu_baseline_block_2k"] = {"value": round(b_ms, 1), "unit": "ms per block",
-                                             "cores": b_threads, "kind": "oracle",
-                                             "estimated": False, "sample": b_desc}
+            def cpu():
+                v, desc, threads, secs = oracle_sample(dh)
+                return {"value": round(v, 1), "unit": "ms", "cores": threads, "kind": "oracle",
+                        "estimated": True, "sample": desc, "sample_cpu_seconds": round(secs, 1)}
+
+            def cpu_2k():
+                b_ms, b_desc, b_threads = oracle_block_2k(dh)
+                return {"value": round(b_ms, 1), "unit": "ms per block", "cores": b_threads,
+                        "kind": "oracle", "estimated": False, "sample": b_desc}
+            line["cpu_baseline"] = optional_leg("cpu_baseline", cpu)
+            line["cpu_baseline_block_2k"] = optional_leg("cpu_baseline_block_2k", cpu_2k)
     # the MXFP8 variant (a11), on the same bf16 weights quantized at create
     if not args.no_mxfp8:
-        from image_generation_b200 import h3dit as Hb
+        def mxfp8():
+            from image_generation_b200 import h3dit as Hb
 
-        cfg_mx = Hb.make_config(D, H, dh, F, L, N_TOK, precision=Hb.H3DIT_PRECISION_MXFP8)
-        ctx_mx = Hb.Context(cfg_mx, tw, blocks)
-        ms_mx, prof_mx, launches_mx = time_steps(ctx_mx, args.steps, args.warmup, x_img, x_txt,
-                                                 grids, barrier, dist)
-        ctx_mx.close()
-        if rank == 0:
+            cfg_mx = Hb.make_config(D, H, dh, F, L, N_TOK, precision=Hb.H3DIT_PRECISION_MXFP8)
+            ctx_mx = Hb.Context(cfg_mx, tw, blocks)
+            ms_mx, prof_mx, launches_mx = time_steps(ctx_mx, args.steps, args.warmup, x_img,
+                                                     x_txt, grids, barrier, dist)
+            ctx_mx.close()
             peaks, peak_src = load_peaks()
             fp8_peak = 2.0 * float(peaks["bf16_tflops_sustained"])
             gemm_kinds = ("qkv", "out_proj", "ffn1", "ffn2")
             gemm_ms = sum(prof_mx[k][0] for k in gemm_kinds)
             gemm_fl = sum(flops_per_launch(k, N_TOK, dh) * prof_mx[k][1] for k in gemm_kinds)
-            mx = {"ms_per_step": round(ms_mx, 2), "value": round(ms_mx / world, 2), "unit": "ms",
-                  "tflops_step": round(step_flops(N_TOK, dh) / ms_mx / 1e9, 1),
-                  "gemm_tflops": round(gemm_fl / gemm_ms / 1e9, 1),
-                  "gemm_frac_of_fp8_peak": round(gemm_fl / gemm_ms / 1e9 / fp8_peak, 4),
-                  "fp8_peak": fp8_peak,
-                  "fp8_peak_source": f"2 x {peak_src} sustained bf16 (nominal fp8:bf16 = 2)",
-                  "kernels": {k: round(v[0] / max(v[1], 1), 4) for k, v in prof_mx.items() if v[1]},
-                  "gpu_launches": launches_mx}
+            g_tf = gemm_fl / gemm_ms / 1e9
+            return {"ms_per_step": round(ms_mx, 2), "value": round(ms_mx / world, 2), "unit": "ms",
+                    "tflops_step": round(step_flops(N_TOK, dh) / ms_mx / 1e9, 1),
+                    "gemm_tflops": round(g_tf, 1),
+                    "gemm_frac_of_fp8_peak": round(g_tf / fp8_peak, 4),
+                    "fp8_peak": fp8_peak,
+                    "fp8_peak_source": f"2 x {peak_src} sustained bf16 (nominal fp8:bf16 = 2)",
+                    "gemm_frac_of_nominal_fp8": round(g_tf / NOMINAL_FP8_TFLOPS, 4),
+                    "kernels": {k: round(v[0] / max(v[1], 1), 4) for k, v in prof_mx.items()
+                                if v[1]},
+                    "gpu_launches": launches_mx}
+        mx = optional_leg("mxfp8", mxfp8)
+        if rank == 0:
             line["mxfp8"] = mx
-            print(json.dumps(line), flush=True)
-    elif rank == 0:
+    if rank == 0:
         print(json.dumps(line), flush=True)
     ctx.close()
     if dist is not None:

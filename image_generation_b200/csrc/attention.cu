@@ -24,7 +24,11 @@
 //               stale max is kept, which leaves O / l unchanged. After the
 //               last tile it normalises O_t by the row sum and stores it.
 // Tensor memory (512 columns): S buffers of tile t at 64 * (2t + b), b = 0, 1;
-// O0 at [256, 256 + d_h), O1 at [384, 384 + d_h).
+// at d_h 128, O0 at [256, 384) and O1 at [384, 512); at d_h 96, O0 at
+// [256, 352), O1 at [352, 448), and the first 64 dimensions of Q_t at
+// [448 + 32 t, 480 + 32 t), written once by the softmax warps in the layout P
+// uses, so that four of the six K16 steps of each S MMA take A from tensor
+// memory instead of re-reading Q from shared memory.
 // Ordering: one thread's MMAs run in issue order; S_t(j+2) is issued after
 // PV_t(j), which read P_t(j) from the same columns, by the same thread. A K/V
 // stage is released once both issuers have committed past its last use.
@@ -48,10 +52,13 @@ constexpr int THREADS = 352;                 // 11 warps
 // P_FULL is per S buffer: with two S buffers a softmax group can finish steps
 // j and j+1 before the MMA warp looks for step j, and a single barrier would
 // then have moved two phases, which a parity wait cannot tell apart.
-constexpr int NUM_BARS = 1 + 2 * NS + 4 + 4 + 2 + 2 + 2;
+constexpr int NUM_BARS = 1 + 2 * NS + 4 + 4 + 2 + 2 + 2 + 2;
 constexpr int SMEM_BYTES = 2 * Q_BYTES + NS * STAGE_BYTES + 1024 + NUM_BARS * 8 + 16;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;    // log2 units
+// d_h 96: Q's first 64 dimensions of tile t live in TMEM at QT_COL + 32 t (A
+// operand of four of the six S MMAs), which moves O_1 to 352.
+constexpr uint32_t QT_COL = 448;
 
 // One row's scores for 64 keys from TMEM; keys at or past `valid` are -inf
 // (only the last KV tile has any).
@@ -123,6 +130,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   constexpr int DCH = (DH + 63) / 64;  // 64-column boxes per row
   constexpr uint32_t IDESC_S = idesc_bf16_f32(BQ, BKV, false, false);
   constexpr uint32_t IDESC_O = idesc_bf16_f32(BQ, DH, false, true);
+  constexpr bool QT = DH == 96;                  // Q (first 64 dims) in TMEM
+  constexpr uint32_t O_STRIDE = QT ? 96 : 128;   // O_t at 256 + O_STRIDE t
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -141,6 +150,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   auto PV_DONE = [&](int t) { return b0 + 8u * (9 + 2 * NS + t); };
   auto O_FULL = [&](int t) { return b0 + 8u * (11 + 2 * NS + t); };
   auto DRAIN = [&](int t) { return b0 + 8u * (13 + 2 * NS + t); };
+  auto Q_TMEM = [&](int t) { return b0 + 8u * (15 + 2 * NS + t); };
 
   __shared__ int aborted;
   if (grid_aborted(p.status, &aborted)) return;
@@ -170,6 +180,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(DRAIN(0), 1);
     mbar_init(DRAIN(1), 1);
+    mbar_init(Q_TMEM(0), 128);
+    mbar_init(Q_TMEM(1), 128);
     fence_mbar_init();
     tma_prefetch_desc(&tq);
     tma_prefetch_desc(&tk);
@@ -213,22 +225,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int t = warp == 1 ? 0 : 1;
       const uint32_t s_base = tmem + 128u * t;
       const uint32_t q_src = sQ + t * Q_BYTES;
-      const uint32_t o_tmem = tmem + 256 + 128 * t;
+      const uint32_t o_tmem = tmem + 256 + O_STRIDE * t;
+      const uint32_t q_tmem = tmem + QT_COL + 32 * t;
       auto issue_s = [&](int j) -> bool {
         if (!mbar_wait(KV_FULL(j % NS), (j / NS) & 1, p.status)) return false;
         tc_fence_after();
         const uint32_t k_src = sKV + (j % NS) * STAGE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
-          umma_bf16(s_base + static_cast<uint32_t>(BKV * (j % SBUF)),
-                    desc_sw128(q_src + (kk / 4) * QBOX + (kk % 4) * 32, 16, 1024),
-                    desc_sw128(k_src + (kk / 4) * KBOX + (kk % 4) * 32, 16, 1024), IDESC_S,
-                    kk > 0 ? 1u : 0u);
+          const uint32_t d = s_base + static_cast<uint32_t>(BKV * (j % SBUF));
+          const uint64_t db = desc_sw128(k_src + (kk / 4) * KBOX + (kk % 4) * 32, 16, 1024);
+          if (QT && kk < 4)
+            umma_bf16_ts(d, q_tmem + 8 * kk, db, IDESC_S, kk > 0 ? 1u : 0u);
+          else
+            umma_bf16(d, desc_sw128(q_src + (kk / 4) * QBOX + (kk % 4) * 32, 16, 1024), db,
+                      IDESC_S, kk > 0 ? 1u : 0u);
         }
         umma_commit(S_FULL(t, j % SBUF));
         return true;
       };
       bool ok = mbar_wait(Q_FULL, 0, p.status);
+      if (QT && ok) {
+        ok = mbar_wait(Q_TMEM(t), 0, p.status);  // the softmax group wrote Q_t into TMEM
+        tc_fence_after();
+      }
       for (int j = 0; j < SBUF && j < nkv && ok; ++j) ok = issue_s(j);
       for (int j = 0; j < nkv && ok; ++j) {
         if (!mbar_wait(P_FULL(t, j % SBUF), (j / SBUF) & 1, p.status)) {
@@ -262,10 +282,31 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int sub = warp & 3;
     const int row = sub * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-    const uint32_t tO = tmem + lane_off + 256 + 128 * t;
+    const uint32_t tO = tmem + lane_off + 256 + O_STRIDE * t;
     const float sl2 = p.scale_log2;
     float m = 0.f, l = 0.f;
     bool ok = true;
+    if (QT) {
+      // this row's first 64 dims of Q (box 0 of the 128-byte-swizzled tile:
+      // 16-byte chunk c of row r at chunk c ^ (r % 8)) into TMEM, packed as
+      // the S MMA's A operand, the layout P is written in
+      ok = mbar_wait(Q_FULL, 0, p.status);
+      if (__all_sync(0xffffffffu, ok)) {
+        const uint8_t *qrow = smem + t * Q_BYTES + row * 128;
+        uint32_t r[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(qrow + ((c ^ (row & 7)) << 4));
+          r[4 * c + 0] = v.x;
+          r[4 * c + 1] = v.y;
+          r[4 * c + 2] = v.z;
+          r[4 * c + 3] = v.w;
+        }
+        tmem_st32(tmem + lane_off + QT_COL + 32 * t, r);
+      }
+      tc_fence_before();
+      mbar_arrive(Q_TMEM(t));  // always, so the issuer's wait ends either way
+    }
     for (int j = 0; j < nkv; ++j) {
       const uint32_t tS = tmem + lane_off + 128u * t + static_cast<uint32_t>(BKV * (j % SBUF));
       ok = mbar_wait(S_FULL(t, j % SBUF), (j / SBUF) & 1, p.status);

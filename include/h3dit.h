@@ -512,8 +512,11 @@ h3dit_status h3dit_attention_batched(h3dit_ctx *ctx, const void *q, const void *
  * that returns H3DIT_ERR_UNSUPPORTED, bad pointers or hidden < 1 or not a
  * multiple of 4 return H3DIT_ERR_INVALID_ARG, both before anything is
  * enqueued. The first call on a device looks up the array's device address
- * for that device (once per device, with it current); make that first call
- * before any stream capture. Every call on a device shares the one array and
+ * for that device (once per device, with it current) and keeps it for the
+ * life of the process; make that first call before any stream capture. A
+ * cudaDeviceReset on a device destroys the array with the context and the
+ * kept address then no longer refers to it, so do not call this entry point
+ * on a device after resetting it. Every call on a device shares the one array and
  * overwrites all of it that it reads, so nothing carries over between calls;
  * two calls that overlap on the GPU (different streams, not ordered) race on
  * it and must be avoided. */
