@@ -5,7 +5,8 @@
 // tcgen05 GEMM with a bias in the epilogue, the attention kernel batched over
 // tiles); this file holds the decoder's own memory-bound steps:
 //   layernorm        (x - mean) / sqrt(var + eps) * gain + bias, fp32 rows in,
-//                    bf16 out; the row stays in registers for both passes
+//                    bf16 out; the row stays in registers for both passes (one
+//                    warp per row up to 2048 wide, one CTA per row beyond)
 //   vae_pos_table    the tile-local 2-D sin-cos position table [T*T, W]
 //   vae_embed        latent [C, Hl, Wl] -> tokens in tile order (tile-major,
 //                    row-major inside a tile): W_in z + b_in + table, fp32
@@ -72,6 +73,54 @@ __global__ void __launch_bounds__(kLnThreads)
 #pragma unroll
     for (int u = 0; u < kLnMaxVec; ++u) {
       const int i = threadIdx.x + u * kLnThreads;
+      if (i < nv) {
+        const float4 g = __ldg(reinterpret_cast<const float4 *>(gain) + i);
+        const float4 b = __ldg(reinterpret_cast<const float4 *>(bias) + i);
+        reinterpret_cast<uint2 *>(out + static_cast<size_t>(row) * d)[i] =
+            make_uint2(pack_bf16x2(fmaf((v[u].x - mean) * rstd, g.x, b.x),
+                                   fmaf((v[u].y - mean) * rstd, g.y, b.y)),
+                       pack_bf16x2(fmaf((v[u].z - mean) * rstd, g.z, b.z),
+                                   fmaf((v[u].w - mean) * rstd, g.w, b.w)));
+      }
+    }
+  }
+}
+
+// Rows of at most 2048 floats: one warp per row, the row in registers (up to
+// 16 float4 per lane), both reductions by shuffles - no block-wide barrier.
+constexpr int kLnWarpMaxVec = 16;
+
+__global__ void __launch_bounds__(256)
+    layernorm_warp_kernel(const float *__restrict__ x, const float *__restrict__ gain,
+                          const float *__restrict__ bias, uint16_t *__restrict__ out, int n, int d,
+                          float eps) {
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const int nv = d / 4;
+  const float inv_d = 1.f / static_cast<float>(d);
+  for (int row = blockIdx.x * warps + (threadIdx.x >> 5); row < n; row += gridDim.x * warps) {
+    const float4 *xr = reinterpret_cast<const float4 *>(x + static_cast<size_t>(row) * d);
+    float4 v[kLnWarpMaxVec];
+    float s = 0.f;
+#pragma unroll
+    for (int u = 0; u < kLnWarpMaxVec; ++u) {
+      const int i = lane + 32 * u;
+      v[u] = i < nv ? __ldcs(xr + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      s += (v[u].x + v[u].y) + (v[u].z + v[u].w);
+    }
+    const float mean = warp_sum_ln(s) * inv_d;
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < kLnWarpMaxVec; ++u) {
+      if (lane + 32 * u < nv) {
+        const float a = v[u].x - mean, b = v[u].y - mean, c = v[u].z - mean, e = v[u].w - mean;
+        ss += (a * a + b * b) + (c * c + e * e);
+      }
+    }
+    const float rstd = rsqrtf(warp_sum_ln(ss) * inv_d + eps);
+#pragma unroll
+    for (int u = 0; u < kLnWarpMaxVec; ++u) {
+      const int i = lane + 32 * u;
       if (i < nv) {
         const float4 g = __ldg(reinterpret_cast<const float4 *>(gain) + i);
         const float4 b = __ldg(reinterpret_cast<const float4 *>(bias) + i);
@@ -203,6 +252,14 @@ int grid_of(long long units, int threads, int num_sms) {
 cudaError_t launch_layernorm(const float *x, const float *gain, const float *bias, void *out,
                              int n, int d, float eps, int num_sms, cudaStream_t s) {
   if (d % 4 || d > 4 * kLnMaxVec * kLnThreads) return cudaErrorInvalidValue;
+  if (d <= 4 * 32 * kLnWarpMaxVec) {
+    const int rows_per_cta = 8;
+    const long long want = (n + rows_per_cta - 1) / rows_per_cta;
+    const int grid = static_cast<int>(want < 16LL * num_sms ? want : 16LL * num_sms);
+    layernorm_warp_kernel<<<grid, 32 * rows_per_cta, 0, s>>>(x, gain, bias,
+                                                              static_cast<uint16_t *>(out), n, d, eps);
+    return cudaGetLastError();
+  }
   const int grid = n < 8 * num_sms ? n : 8 * num_sms;
   layernorm_kernel<<<grid, kLnThreads, 0, s>>>(x, gain, bias, static_cast<uint16_t *>(out), n, d,
                                                eps);

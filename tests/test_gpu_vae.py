@@ -155,3 +155,25 @@ def test_decode_writes_only_the_image_and_rejects_bad_shapes(small):
         ctx.time_embed(0.5, torch.empty(256, device="cuda"))
     assert e.value.status == H.H3DIT_ERR_UNSUPPORTED
     _ok(ctx)
+
+
+@pytest.mark.parametrize("n", [1, 300])
+def test_layernorm_wide_rows(n):
+    """Rows wider than 2048 take the one-CTA-per-row form (a full-width DiT
+    context, width 5376)."""
+    from image_generation_b200 import h3dit as H
+    from tests.helpers import time_tensors
+
+    d = synth.FULL_96
+    bw = {k: torch.zeros(16, device="cuda", dtype=torch.bfloat16)
+          for k in ("w_qkv", "w_o", "w_ff1", "w_ff2", "w_ada")}
+    bw["b_ada"] = torch.zeros(16, device="cuda")
+    ctx = H.Context(H.make_config(d.hidden, d.heads, d.head_dim, d.ffn, 1, 16),
+                    time_tensors(synth.time_weights(d, 0)), [bw])
+    x = synth.normal_f32((n, d.hidden), 2.0, n, "xw") - 0.4
+    g = (1.0 + synth.normal_f32((d.hidden,), 0.1, n, "g")).astype(np.float32)
+    b = synth.normal_f32((d.hidden,), 0.1, n, "b")
+    out = torch.empty(n, d.hidden, dtype=torch.bfloat16, device="cuda")
+    ctx.layernorm(to_dev(x, "f32"), to_dev(g, "f32"), to_dev(b, "f32"), out)
+    _ok(ctx)
+    assert_bf16_rounding(to_np(out), V.layer_norm(x, g, b, 1e-6), "wide layernorm", abs_floor=1e-4)
