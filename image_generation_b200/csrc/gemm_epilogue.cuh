@@ -14,7 +14,10 @@
 namespace h3 {
 namespace gemm_detail {
 
-constexpr int GROUP_M = 16;
+#ifndef H3_GEMM_GROUP_M
+#define H3_GEMM_GROUP_M 16
+#endif
+constexpr int GROUP_M = H3_GEMM_GROUP_M;
 
 // Grouped raster: GROUP_M row-tiles sweep all column tiles together so that
 // the CTAs running at once share A and W tiles in L2.
