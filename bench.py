@@ -54,7 +54,8 @@ def parse():
     ap.add_argument("--impl", default="h3dit", choices=["h3dit", "reference"])
     ap.add_argument("--head-dim", type=int, default=96, choices=[96, 128])
     ap.add_argument("--only", default=None,
-                    choices=["attention", "qkv", "out_proj", "ffn1", "ffn2", "rmsnorm", "adaln"])
+                    choices=["attention", "qkv", "out_proj", "ffn1", "ffn2", "rmsnorm", "adaln",
+                             "vae"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-mxfp8", action="store_true")
@@ -455,10 +456,16 @@ def run_reference(args):
 
 
 def run_only(args):
-    """One kernel kind alone at the step's shape (for ncu captures)."""
+    """One kernel kind alone at the step's shape (for ncu captures); "vae" is
+    the VAE decoder on the 4096^2 canvas's latent, --warmup + --steps decodes."""
     import torch
 
     from image_generation_b200 import h3dit as Hb
+
+    if args.only == "vae":
+        out = vae_timing(reps=max(args.steps, 1), warmup=args.warmup, graph=False)
+        print(json.dumps({"kernel": "vae_decode", **out}), flush=True)
+        return 0
 
     dh = args.head_dim
     I = H * dh
@@ -658,7 +665,7 @@ def vae_flops(n_tok: int, tile: int, W=1280, M=5120, layers=24, C=24) -> float:
     return float(lin + layers * (n_tok // n) * 4 * n * n * W)
 
 
-def vae_timing(reps: int = 5) -> dict:
+def vae_timing(reps: int = 5, warmup: int = 2, graph: bool = True) -> dict:
     """The image VAE's 24-layer ViT decoder (width 1280, 10 heads x 128, MLP
     5120, 32 x 32 latent tiles) decoding the 4096^2 canvas's latent
     [24, 256, 256] (64 tiles, 65,536 tokens) on random device weights: ms per
@@ -684,7 +691,7 @@ def vae_timing(reps: int = 5) -> dict:
     dec = Hb.VaeDecoder(cfg, weights)
     z = torch.randn(24, hl, hl, device="cuda", generator=g)
     img = torch.empty(3, 16 * hl, 16 * hl, device="cuda")
-    for _ in range(2):
+    for _ in range(warmup):
         dec.decode(z, img)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -696,25 +703,28 @@ def vae_timing(reps: int = 5) -> dict:
     torch.cuda.synchronize()
     prof = dec.profile_end()
     ms = e0.elapsed_time(e1) / reps
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        dec.decode(z, img)
-    graph.replay()
-    torch.cuda.synchronize()
-    e0.record()
-    for _ in range(reps):
-        graph.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    g_ms = e0.elapsed_time(e1) / reps
-    del graph
+    g_ms = None
+    if graph:
+        cg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cg):
+            dec.decode(z, img)
+        cg.replay()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            cg.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        g_ms = e0.elapsed_time(e1) / reps
+        del cg
     if dec.sync_status() != 0 or not bool(torch.isfinite(img).all()):
         raise RuntimeError("VAE decode failed")
     fl = vae_flops(hl * hl, T)
     tot = sum(v[0] for v in prof.values()) or 1.0
     att_ms, att_n = prof["attention"]
     att_fl = L_ * (hl * hl // (T * T)) * 4.0 * (T * T) ** 2 * W
-    out = {"ms": round(ms, 2), "graph_ms": round(g_ms, 2), "tokens": hl * hl,
+    out = {"ms": round(ms, 2), "graph_ms": None if g_ms is None else round(g_ms, 2),
+           "tokens": hl * hl,
            "tiles": hl * hl // (T * T), "image": [3, 16 * hl, 16 * hl],
            "tflops": round(fl / ms / 1e9, 1),
            "attention_tflops": round(att_fl * reps / att_ms / 1e9, 1) if att_n else None,

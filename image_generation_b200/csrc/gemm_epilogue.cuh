@@ -153,10 +153,14 @@ __device__ __forceinline__ void plain_chunk(const GemmParams &p, uint32_t taddr,
   }
 }
 
+// part / parts: the thread handles every parts-th unit (32 columns, or a
+// rotary section) of the tile starting at unit `part`, so several epilogue
+// warps on one TMEM lane quarter can share a tile.
 template <int EPI, int BN>
 __device__ __forceinline__ void epilogue_tile(const GemmParams &p, uint32_t tbase, int row,
-                                              int col_tile) {
+                                              int col_tile, int part = 0, int parts = 1) {
   const bool row_ok = row < p.m;
+  int unit = 0;
   if constexpr (EPI == kEpiQkvRope) {
     int c = 0;
     while (c < BN) {
@@ -175,21 +179,22 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, uint32_t tbas
           s = p.sec[2];
           pb = p.sec[0] + p.sec[1];
         }
+        const bool mine = unit++ % parts == part;
         if (s == 16) {
-          rope_unit<16>(p, tbase + c, row, col, pb, row_ok);
+          if (mine) rope_unit<16>(p, tbase + c, row, col, pb, row_ok);
           c += 32;
         } else {
-          rope_unit<24>(p, tbase + c, row, col, pb, row_ok);
+          if (mine) rope_unit<24>(p, tbase + c, row, col, pb, row_ok);
           c += 48;
         }
       } else {
-        plain_chunk<kEpiStore>(p, tbase + c, row, col, row_ok);
+        if (unit++ % parts == part) plain_chunk<kEpiStore>(p, tbase + c, row, col, row_ok);
         c += 32;
       }
     }
   } else {
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = 32 * part; c < BN; c += 32 * parts) {
       const int col = col_tile + c;
       if (col >= p.n) break;
       plain_chunk<EPI>(p, tbase + c, row, col, row_ok);

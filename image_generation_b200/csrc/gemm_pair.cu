@@ -18,7 +18,11 @@
 //               issuer: 4 pair MMAs per k-block into one of two 256-column
 //               accumulators; each commit arrives on both CTAs' EMPTY / TFULL;
 //   warps 2..5  epilogue of this CTA's 128 rows, unchanged from the one-CTA
-//               kernel; every thread then arrives on the first CTA's TEMPTY.
+//   (..9)       kernel; every thread then arrives on the first CTA's TEMPTY.
+//               With PARTS = 2 (launches whose K is at most 2048, where a
+//               tile's mainloop is short next to a GELU or residual epilogue),
+//               eight warps share it, two per TMEM lane quarter, each taking
+//               every other 32-column unit of the tile.
 //
 // The decision to skip work after an earlier failure is taken for the pair
 // as a whole, and a CTA leaves only after both producers' loads have landed,
@@ -39,15 +43,18 @@ constexpr int STAGES = 6;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = (BN / 2) * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int THREADS = 192;
+template <int PARTS>
+constexpr int threads_for() {
+  return 64 + 128 * PARTS;
+}
 constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + NUM_BARS * 8 + 16;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC = idesc_bf16_f32(2 * BM, BN, false, false);
 constexpr uint16_t kBothCtas = 0x3, kFirstCta = 0x1;
 
-template <int EPI>
-__global__ void __launch_bounds__(THREADS, 1)
+template <int EPI, int PARTS>
+__global__ void __launch_bounds__(threads_for<PARTS>(), 1)
     gemm_bf16_pair(const __grid_constant__ CUtensorMap tma_a,
                    const __grid_constant__ CUtensorMap tma_b, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -80,7 +87,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(TFULL(a), 1);
-      mbar_init(TEMPTY(a), 2 * 128);  // both CTAs' epilogue threads
+      mbar_init(TEMPTY(a), 2 * 128 * PARTS);  // both CTAs' epilogue threads
     }
     mbar_init(DRAIN, 1);
     fence_mbar_init();
@@ -199,7 +206,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t tbase =
           tmem + (static_cast<uint32_t>(sub * 32) << 16) + static_cast<uint32_t>(acc * BN);
       epilogue_tile<EPI, BN>(p, tbase, tm * 2 * BM + static_cast<int>(rank) * BM + row_in_tile,
-                             tn * BN);
+                             tn * BN, (warp - 2) >> 2, PARTS);
       tc_fence_before();
       if (leader)
         mbar_arrive(TEMPTY(acc));
@@ -235,15 +242,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int EPI>
+template <int EPI, int PARTS>
 cudaError_t launch_one(const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p, int grid,
                        cudaStream_t s) {
   static PerDevice smem_attr;
-  cudaError_t e = set_smem_once(smem_attr, gemm_bf16_pair<EPI>, SMEM_BYTES);
+  cudaError_t e = set_smem_once(smem_attr, gemm_bf16_pair<EPI, PARTS>, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.blockDim = dim3(threads_for<PARTS>(), 1, 1);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -253,7 +260,14 @@ cudaError_t launch_one(const CUtensorMap &a, const CUtensorMap &b, const GemmPar
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_bf16_pair<EPI>, a, b, p);
+  return cudaLaunchKernelEx(&cfg, gemm_bf16_pair<EPI, PARTS>, a, b, p);
+}
+
+// The epilogue on eight warps where the mainloop is short (K <= 2048).
+template <int EPI>
+cudaError_t launch_parts(const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p, int grid,
+                         cudaStream_t s) {
+  return p.k <= 2048 ? launch_one<EPI, 2>(a, b, p, grid, s) : launch_one<EPI, 1>(a, b, p, grid, s);
 }
 
 template <int EPI>
@@ -267,7 +281,8 @@ int max_pairs_for() {
   int n = 0;
   if (per_device(pairs, [](int *v) {
         *v = 0;
-        if (cudaFuncSetAttribute(gemm_bf16_pair<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        // both forms hold one CTA per SM (the same shared memory)
+        if (cudaFuncSetAttribute(gemm_bf16_pair<EPI, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  SMEM_BYTES) != cudaSuccess) {
           cudaGetLastError();
           return cudaSuccess;
@@ -283,7 +298,7 @@ template <int EPI>
 int occupancy_clusters() {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(2, 1, 1);
-  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.blockDim = dim3(threads_for<1>(), 1, 1);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -293,7 +308,7 @@ int occupancy_clusters() {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_bf16_pair<EPI>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_bf16_pair<EPI, 1>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     n = 0;
   }
@@ -322,13 +337,13 @@ cudaError_t launch_gemm_pair(const CUtensorMap &a, const CUtensorMap &b, const G
   if (grid <= 0 || (grid & 1)) return cudaErrorInvalidValue;
   switch (epilogue) {
     case kEpiStore:
-      return launch_one<kEpiStore>(a, b, p, grid, s);
+      return launch_parts<kEpiStore>(a, b, p, grid, s);
     case kEpiQkvRope:
-      return launch_one<kEpiQkvRope>(a, b, p, grid, s);
+      return launch_parts<kEpiQkvRope>(a, b, p, grid, s);
     case kEpiGelu:
-      return launch_one<kEpiGelu>(a, b, p, grid, s);
+      return launch_parts<kEpiGelu>(a, b, p, grid, s);
     case kEpiGatedResidual:
-      return launch_one<kEpiGatedResidual>(a, b, p, grid, s);
+      return launch_parts<kEpiGatedResidual>(a, b, p, grid, s);
     default:
       return cudaErrorInvalidValue;
   }

@@ -473,6 +473,8 @@ class VaeDecoder(Context):
             raise H3DitError(H3DIT_ERR_INVALID_ARG, "invalid decoder config")
         if workspace is None:
             workspace = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        elif workspace.numel() * workspace.element_size() < ws_bytes:
+            raise H3DitError(H3DIT_ERR_WORKSPACE, "workspace smaller than h3dit_vae_workspace_bytes")
         self.workspace = workspace
         names = [f[0] for f in h3dit_vae_layer_weights._fields_]
         layers = (h3dit_vae_layer_weights * len(weights["layers"]))()

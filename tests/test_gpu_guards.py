@@ -279,3 +279,68 @@ def test_time_embed_static():
                                        torch.cuda.current_stream().cuda_stream)
     assert st == H.H3DIT_OK
     c.check("static time embed")
+
+
+@pytest.mark.parametrize("P", [2, 4])
+def test_sequence_parallel_relayouts(bf16_ctx, P):
+    ctx, ws, _ = bf16_ctx
+    I = synth.SMALL.inner
+    n = 37  # rows of one rank, not a multiple of anything
+    qkv = torch.randn(n, 3 * I, device="cuda").bfloat16()
+    send = Guarded((P, n, 3 * I // P), torch.bfloat16)
+    ctx.sp_pack_qkv(qkv, P, send.t)
+    send.check(f"sequence-parallel pack, {P} ranks")
+    recv = torch.randn(P, n, I // P, device="cuda").bfloat16()
+    o = Guarded((n, I), torch.bfloat16)
+    ctx.sp_unpack_o(recv, P, o.t)
+    o.check(f"sequence-parallel unpack, {P} ranks")
+    heads = synth.SMALL.heads // P
+    q = torch.randn(P * n, 3 * I // P, device="cuda").bfloat16()
+    cw = I // P
+    oh = Guarded((P * n, cw + 16), torch.bfloat16)   # rows wider than the head group
+    ctx.attention_heads(heads, q[:, :cw], q[:, cw:2 * cw], q[:, 2 * cw:], 3 * cw, oh.t, cw + 16,
+                        P * n)
+    oh.check(f"attention on {heads} heads")
+    torch.cuda.synchronize()
+    assert bool((oh.t[:, cw:].contiguous().view(torch.uint8) == 0xFF).all())
+    _ok(ctx, ws, f"sequence-parallel {P}")
+
+
+@pytest.mark.parametrize("m", [1, 130, 257])
+def test_decoder_stage_entry_points(m):
+    from image_generation_b200 import h3dit as H
+
+    import ctypes as C
+
+    v = synth.VAE_SMALL
+    cfg = H.make_vae_config(v.width, v.heads, v.head_dim, v.mlp, v.layers, v.tile, v.channels,
+                            2048)
+    ws = Guarded((int(H.lib.h3dit_vae_workspace_bytes(C.byref(cfg))),), torch.uint8)
+    w = synth.vae_weights(v, 0)
+    dev = {k: to_dev(val, "bf16" if k == "w_out" else "f32") for k, val in w.items()
+           if k != "layers"}
+    mats = ("w_qkv", "w_o", "w_1", "w_2")
+    dev["layers"] = [{k: to_dev(val, "bf16" if k in mats else "f32") for k, val in l.items()}
+                     for l in w["layers"]]
+    ctx = H.VaeDecoder(cfg, dev, workspace=ws.t)
+    W = v.width
+    x = torch.randn(m, W, device="cuda")
+    ln = Guarded((m, W), torch.bfloat16)
+    ctx.layernorm(x, dev["lnf_g"], dev["lnf_b"], ln.t)
+    ln.check(f"layernorm m={m}")
+    wt = torch.randn(800, W, device="cuda").bfloat16()
+    b = torch.randn(800, device="cuda")
+    for epi in (H.H3DIT_EPI_STORE, H.H3DIT_EPI_GELU):
+        out = Guarded((m, 800), torch.bfloat16)
+        ctx.linear_bias(epi, ln.t, wt, b, out.t)
+        out.check(f"linear + bias, epilogue {epi}, m={m}")
+    res = Guarded((m, 800), torch.float32, init=torch.randn(m, 800, device="cuda"))
+    ctx.linear_bias(H.H3DIT_EPI_GATED_RESIDUAL, ln.t, wt, b, res.t,
+                    gate=torch.ones(800, device="cuda"))
+    res.check(f"residual + linear + bias, m={m}")
+    I = v.heads * v.head_dim
+    q = torch.randn(3 * m, 3 * I, device="cuda").bfloat16()
+    o = Guarded((3 * m, I), torch.bfloat16)
+    ctx.attention_batched(q[:, :I], q[:, I:2 * I], q[:, 2 * I:], 3 * I, o.t, I, m, 3)
+    o.check(f"attention over 3 sequences of {m}")
+    _ok(ctx, ws, f"decoder stages m={m}")
