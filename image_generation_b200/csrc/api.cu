@@ -368,15 +368,22 @@ h3dit_status encode_heads(h3dit_ctx *ctx, CUtensorMap *m, const void *base, int 
   return H3DIT_OK;
 }
 
+// Destination buffers of a fused Ulysses exchange, one per rank.
+struct ScatterTargets {
+  void *const *ptr;
+  int ranks, rank;
+};
+
 h3dit_status run_linear(h3dit_ctx *ctx, int epi, const void *a, const void *w, int m, int n,
                         int k, void *out, long long ldo, const float *gate, const float *rope,
-                        cudaStream_t s, const float *bias = nullptr, int kind_override = -1) {
+                        cudaStream_t s, const float *bias = nullptr, int kind_override = -1,
+                        const ScatterTargets *scatter = nullptr) {
   if (epi < H3DIT_EPI_STORE || epi > H3DIT_EPI_GATED_RESIDUAL)
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "unknown epilogue %d", epi);
   if (m < 0 || n <= 0 || k <= 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "bad shape %d x %d x %d", m, n, k);
   if (k % kGemmBK || n % 32)
     return ctx->fail(H3DIT_ERR_UNSUPPORTED, "linear needs k %% 64 == 0 and n %% 32 == 0 (k=%d n=%d)", k, n);
-  if (!a || !w || !out || !aligned16(a) || !aligned16(w) || !aligned16(out))
+  if (!a || !w || (!scatter && (!out || !aligned16(out))) || !aligned16(a) || !aligned16(w))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "linear: NULL or misaligned pointer");
   if (epi == H3DIT_EPI_GATED_RESIDUAL && (!gate || !aligned16(gate)))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "gated residual needs a 16-byte aligned gate");
@@ -400,6 +407,16 @@ h3dit_status run_linear(h3dit_ctx *ctx, int epi, const void *a, const void *w, i
     p.sec[0] = sec[0];
     p.sec[1] = sec[1];
     p.sec[2] = sec[2];
+    if (scatter) {
+      // each rank's receive buffer is [ranks * m, 3 * I / ranks]; every
+      // 32- or 48-column store unit sits in one head and starts on a
+      // multiple of 8 columns, so the 16-byte stores stay aligned
+      p.scatter_ranks = scatter->ranks;
+      p.scatter_rank = scatter->rank;
+      p.scatter_inner = I;
+      p.scatter_cols = I / scatter->ranks;
+      for (int g = 0; g < scatter->ranks; ++g) p.scatter[g] = scatter->ptr[g];
+    }
   }
   if (m == 0) return H3DIT_OK;
   // More than one 128-row block: 256 x 256 tiles on CTA pairs, which halves
@@ -530,14 +547,16 @@ h3dit_status run_linear_mx(h3dit_ctx *ctx, int epi, const void *a, const void *a
 
 h3dit_status run_attention(h3dit_ctx *ctx, const void *q, const void *k, const void *v, int ld,
                            void *o, int ldo, int n, cudaStream_t s, void *o_sf = nullptr,
-                           int heads = 0, int batch = 1) {
+                           int heads = 0, int batch = 1,
+                           const ScatterTargets *scatter = nullptr) {
   if (heads == 0) heads = ctx->cfg.heads;
   if (n < 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "n < 0");
   if (batch < 1 || static_cast<long long>(n) * batch > (1LL << 30))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "bad sequence batch");
   if (heads < 1 || heads > ctx->cfg.heads)
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "heads %d outside [1, %d]", heads, ctx->cfg.heads);
-  if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+  if (!q || !k || !v || (!scatter && (!o || !aligned16(o))) || !aligned16(q) || !aligned16(k) ||
+      !aligned16(v))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "attention: NULL or misaligned pointer");
   const int I = heads * ctx->cfg.head_dim;
   if (ld < I || ld % 8 || ldo < I || ldo % 8)
@@ -560,6 +579,14 @@ h3dit_status run_attention(h3dit_ctx *ctx, const void *q, const void *k, const v
   p.o_sf = static_cast<uint8_t *>(o_sf);
   if (o_sf && (ldo != I || I % 128 || !aligned16(o_sf)))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "MXFP8 attention output needs ld_o == heads*head_dim, a multiple of 128");
+  if (scatter) {
+    // rank r's rows of the sequence go to its [n / ranks, ld_o] output, at
+    // this rank's head group's columns
+    p.o_scatter_ranks = scatter->ranks;
+    p.o_rows_per_rank = n / scatter->ranks;
+    p.o_col0 = scatter->rank * I;
+    for (int g = 0; g < scatter->ranks; ++g) p.o_scatter[g] = scatter->ptr[g];
+  }
   Launch L(ctx, H3DIT_KERNEL_ATTENTION, s);
   return ctx->cuda(launch_attention(tq, tk, tv, p, ctx->cfg.head_dim, heads, o_sf != nullptr, s),
                    "attention launch");
@@ -1188,6 +1215,111 @@ h3dit_status h3dit_sp_unpack_o(h3dit_ctx *ctx, const void *recv, int32_t n_local
   return ctx->cuda(launch_sp_unpack_o(recv, n_local, ranks, ctx->inner() / ranks, o, ctx->num_sms,
                                       s),
                    "sequence parallel unpack launch");
+}
+
+namespace {
+h3dit_status check_scatter(h3dit_ctx *ctx, void *const *dst, int ranks, int rank) {
+  if (ranks < 1 || ranks > kMaxScatterRanks)
+    return ctx->fail(H3DIT_ERR_UNSUPPORTED, "%d ranks: the fused exchange addresses 1 .. %d",
+                     ranks, kMaxScatterRanks);
+  if (rank < 0 || rank >= ranks)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "rank %d outside [0, %d)", rank, ranks);
+  if (!dst) return ctx->fail(H3DIT_ERR_INVALID_ARG, "NULL destination array");
+  for (int g = 0; g < ranks; ++g)
+    if (!dst[g] || !aligned16(dst[g]))
+      return ctx->fail(H3DIT_ERR_INVALID_ARG, "destination of rank %d is NULL or misaligned", g);
+  return H3DIT_OK;
+}
+}  // namespace
+
+h3dit_status h3dit_sp_qkv_scatter(h3dit_ctx *ctx, const void *xm, int32_t n_local,
+                                  const void *w_qkv, const float *rope_rows, void *const *recv,
+                                  int32_t ranks, int32_t rank, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (ctx->vae) return ctx->fail(H3DIT_ERR_UNSUPPORTED, "a decoder context runs h3dit_vae_decode");
+  h3dit_status st = check_scatter(ctx, recv, ranks, rank);
+  if (st) return st;
+  if ((st = check_sp(ctx, xm, w_qkv, n_local, ranks))) return st;
+  const ScatterTargets sc{recv, ranks, rank};
+  const int I = ctx->inner();
+  return run_linear(ctx, H3DIT_EPI_QKV_ROPE, xm, w_qkv, n_local, 3 * I, ctx->cfg.hidden, nullptr,
+                    0, nullptr, rope_rows, static_cast<cudaStream_t>(cuda_stream), nullptr, -1,
+                    &sc);
+}
+
+h3dit_status h3dit_sp_attention_scatter(h3dit_ctx *ctx, const void *qkv, int32_t n_total,
+                                        void *const *o, int32_t ranks, int32_t rank,
+                                        void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (ctx->vae) return ctx->fail(H3DIT_ERR_UNSUPPORTED, "a decoder context runs h3dit_vae_decode");
+  h3dit_status st = check_scatter(ctx, o, ranks, rank);
+  if (st) return st;
+  if ((st = check_sp(ctx, qkv, o[0], n_total, ranks))) return st;
+  if (n_total % ranks)
+    return ctx->fail(H3DIT_ERR_UNSUPPORTED, "%d tokens do not split over %d ranks", n_total, ranks);
+  const ScatterTargets sc{o, ranks, rank};
+  const int I = ctx->inner(), cw = I / ranks;
+  const uint16_t *q = static_cast<const uint16_t *>(qkv);
+  return run_attention(ctx, q, q + cw, q + 2 * cw, 3 * cw, nullptr, I, n_total,
+                       static_cast<cudaStream_t>(cuda_stream), nullptr, ctx->cfg.heads / ranks, 1,
+                       &sc);
+}
+
+namespace {
+typedef CUresult (*AddressRangeFn)(CUdeviceptr *, size_t *, CUdeviceptr);
+AddressRangeFn address_range_fn() {
+  static AddressRangeFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<AddressRangeFn>(p);
+  }
+  return fn;
+}
+}  // namespace
+
+h3dit_status h3dit_ipc_get_handle(const void *dev_ptr, void *handle_out, uint64_t *offset_out) {
+  static_assert(sizeof(cudaIpcMemHandle_t) == H3DIT_IPC_HANDLE_BYTES, "IPC handle size");
+  if (!dev_ptr || !handle_out || !offset_out) return H3DIT_ERR_INVALID_ARG;
+  AddressRangeFn range = address_range_fn();
+  if (!range) return H3DIT_ERR_CUDA;
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (range(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS)
+    return H3DIT_ERR_CUDA;
+  cudaIpcMemHandle_t h;
+  if (cudaIpcGetMemHandle(&h, reinterpret_cast<void *>(base)) != cudaSuccess) {
+    cudaGetLastError();
+    return H3DIT_ERR_CUDA;
+  }
+  std::memcpy(handle_out, &h, sizeof h);
+  *offset_out = reinterpret_cast<uintptr_t>(dev_ptr) - static_cast<uintptr_t>(base);
+  return H3DIT_OK;
+}
+
+h3dit_status h3dit_ipc_open(const void *handle, uint64_t offset, void **dev_ptr_out) {
+  if (!handle || !dev_ptr_out) return H3DIT_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  std::memcpy(&h, handle, sizeof h);
+  void *base = nullptr;
+  if (cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+    cudaGetLastError();
+    return H3DIT_ERR_CUDA;
+  }
+  *dev_ptr_out = static_cast<uint8_t *>(base) + offset;
+  return H3DIT_OK;
+}
+
+h3dit_status h3dit_ipc_close(void *dev_ptr, uint64_t offset) {
+  if (!dev_ptr) return H3DIT_ERR_INVALID_ARG;
+  if (cudaIpcCloseMemHandle(static_cast<uint8_t *>(dev_ptr) - offset) != cudaSuccess) {
+    cudaGetLastError();
+    return H3DIT_ERR_CUDA;
+  }
+  return H3DIT_OK;
 }
 
 h3dit_status h3dit_block_forward(h3dit_ctx *ctx, int32_t block, float t, const float *mod,

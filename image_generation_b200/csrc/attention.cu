@@ -371,7 +371,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float inv_l = 1.f / l;
       const int qrow = q0 + t * BQ + row;  // within the sequence
       const size_t grow = static_cast<size_t>(seq0) + qrow;
-      uint16_t *dst = static_cast<uint16_t *>(p.o) + grow * p.ldo + head * DH;
+      uint16_t *dst;
+      if (p.o_scatter_ranks == 0) {
+        dst = static_cast<uint16_t *>(p.o) + grow * p.ldo + head * DH;
+      } else {
+        // the second Ulysses all-to-all: this row belongs to rank grow / rows
+        const int owner = static_cast<int>(grow / static_cast<size_t>(p.o_rows_per_rank));
+        const size_t local = grow - static_cast<size_t>(owner) * p.o_rows_per_rank;
+        dst = static_cast<uint16_t *>(p.o_scatter[owner < kMaxScatterRanks ? owner : 0]) +
+              local * p.ldo + p.o_col0 + head * DH;
+      }
 #pragma unroll
       for (int c = 0; c < DH / 32; ++c) {
         uint32_t r[32];

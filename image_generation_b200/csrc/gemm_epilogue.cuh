@@ -69,6 +69,22 @@ __device__ __forceinline__ void store_bf16_row(void *dst, const float *v) {
   }
 }
 
+// Where the bf16 output element (row, col) goes: the row-major output, or,
+// with the first Ulysses all-to-all fused into QKV + RoPE, the receive buffer
+// of the rank that attends over col's head group, at this rank's block of
+// sequence rows. A store unit (32 columns, or one rotary section) lies inside
+// one head, so it goes to one rank and stays contiguous there.
+__device__ __forceinline__ uint16_t *out_bf16(const GemmParams &p, int row, int col) {
+  if (p.scatter_ranks == 0)
+    return static_cast<uint16_t *>(p.out) + static_cast<size_t>(row) * p.ldo + col;
+  const int q = col / p.scatter_inner;  // 0 Q, 1 K, 2 V
+  const int c = col - q * p.scatter_inner;
+  const int g = c / p.scatter_cols;     // head group = destination rank
+  const size_t r = static_cast<size_t>(p.scatter_rank) * p.m + row;
+  return static_cast<uint16_t *>(p.scatter[g]) + r * (3 * p.scatter_cols) + q * p.scatter_cols +
+         (c - g * p.scatter_cols);
+}
+
 // One rotary unit: 2*S accumulator columns holding S rotation pairs (j, S + j).
 template <int S>
 __device__ __forceinline__ void rope_unit(const GemmParams &p, uint32_t taddr, int row, int col,
@@ -98,7 +114,7 @@ __device__ __forceinline__ void rope_unit(const GemmParams &p, uint32_t taddr, i
     v[j + 1] = a1 * t.z - b1 * t.w;
     v[S + j + 1] = b1 * t.z + a1 * t.w;
   }
-  store_bf16_row<2 * S>(static_cast<uint16_t *>(p.out) + static_cast<size_t>(row) * p.ldo + col, v);
+  store_bf16_row<2 * S>(out_bf16(p, row, col), v);
 }
 
 template <int EPI>
@@ -149,7 +165,7 @@ __device__ __forceinline__ void plain_chunk(const GemmParams &p, uint32_t taddr,
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] = gelu_f(v[i], p.gelu_tanh);
     }
-    store_bf16_row<32>(static_cast<uint16_t *>(p.out) + static_cast<size_t>(row) * p.ldo + col, v);
+    store_bf16_row<32>(out_bf16(p, row, col), v);
   }
 }
 

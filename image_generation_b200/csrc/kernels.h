@@ -78,6 +78,10 @@ inline size_t mx_sf_bytes(long long rows, long long k) {
   return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>(k / 128) * 512;
 }
 
+// Ranks a fused Ulysses exchange can address (destination pointers carried
+// in the kernel parameters).
+constexpr int kMaxScatterRanks = 8;
+
 struct GemmParams {
   int m, n, k;
   int tiles_m, tiles_n;
@@ -94,6 +98,15 @@ struct GemmParams {
   // MXFP8 only
   const uint8_t *a_sf, *b_sf;  // scale factors of A [m, k] and W [n, k]
   uint8_t *out_sf;             // GELU-MXFP8 epilogue: scales of out [m, n]
+  // QKV + RoPE with the first Ulysses all-to-all fused in (scatter_ranks > 0):
+  // column c of matrix q (0 Q, 1 K, 2 V) in head group g = c / scatter_cols
+  // of output row r goes to scatter[g] at row scatter_rank * m + r, column
+  // q * scatter_cols + c % scatter_cols, of a [ranks * m, 3 * scatter_cols]
+  // bf16 buffer; `out` is unused.
+  void *scatter[kMaxScatterRanks];
+  int scatter_ranks, scatter_rank;
+  int scatter_inner;           // heads * head_dim (width of one of Q, K, V)
+  int scatter_cols;            // columns of one head group
 };
 
 struct AttnParams {
@@ -105,6 +118,13 @@ struct AttnParams {
   float scale_log2;       // log2(e) / sqrt(head_dim)
   int *status;
   uint8_t *o_sf;          // MXFP8 output: scales of o [n, heads*head_dim]
+  // The second Ulysses all-to-all fused in (o_scatter_ranks > 0): output row
+  // t goes to o_scatter[t / o_rows_per_rank] at row t % o_rows_per_rank,
+  // column o_col0 + head * head_dim, with row stride ldo; `o` is unused.
+  void *o_scatter[kMaxScatterRanks];
+  int o_scatter_ranks;
+  int o_rows_per_rank;
+  int o_col0;
 };
 
 // Tile of the tcgen05 GEMM (rows x columns of the output).

@@ -36,6 +36,8 @@ H3DIT_LINEAR_FFN2 = 3
 H3DIT_PRECISION_BF16 = 0
 H3DIT_PRECISION_MXFP8 = 1
 H3DIT_STATIC_TIME_MAX_HIDDEN = 8192
+H3DIT_MAX_SCATTER_RANKS = 8
+H3DIT_IPC_HANDLE_BYTES = 64
 
 KERNEL_KINDS = ["time_embed", "adaln", "rmsnorm", "qkv", "attention", "out_proj", "ffn1",
                 "ffn2", "rope_table", "pack", "mx_quantize", "io"]
@@ -130,6 +132,11 @@ def _load() -> C.CDLL:
         "h3dit_attention_heads": (i32, [p, i32, p, p, p, i32, p, i32, i32, p]),
         "h3dit_sp_pack_qkv": (i32, [p, p, i32, i32, p, p]),
         "h3dit_sp_unpack_o": (i32, [p, p, i32, i32, p, p]),
+        "h3dit_sp_qkv_scatter": (i32, [p, p, i32, p, p, C.POINTER(p), i32, i32, p]),
+        "h3dit_sp_attention_scatter": (i32, [p, p, i32, C.POINTER(p), i32, i32, p]),
+        "h3dit_ipc_get_handle": (i32, [p, p, C.POINTER(C.c_uint64)]),
+        "h3dit_ipc_open": (i32, [p, C.c_uint64, C.POINTER(p)]),
+        "h3dit_ipc_close": (i32, [p, C.c_uint64]),
         "h3dit_vae_workspace_bytes": (sz, [C.POINTER(h3dit_vae_config)]),
         "h3dit_vae_create": (i32, [C.POINTER(h3dit_vae_config), C.POINTER(h3dit_vae_weights), p,
                                    sz, p, C.POINTER(p)]),
@@ -235,6 +242,29 @@ def _stream(stream=None) -> int:
 
     s = stream if stream is not None else torch.cuda.current_stream()
     return s.cuda_stream
+
+
+def ipc_handle(t) -> Tuple[bytes, int]:
+    """(handle, offset) naming the device memory of tensor t for another
+    process on this node (CUDA IPC; see h3dit_ipc_get_handle)."""
+    h = (C.c_char * H3DIT_IPC_HANDLE_BYTES)()
+    off = C.c_uint64()
+    check(None, lib.h3dit_ipc_get_handle(_ptr(t, False), h, C.byref(off)))
+    return bytes(h), int(off.value)
+
+
+def ipc_open(handle: bytes, offset: int) -> int:
+    """Device address, in this process, of the byte another process named
+    with ipc_handle."""
+    if len(handle) != H3DIT_IPC_HANDLE_BYTES:
+        raise H3DitError(H3DIT_ERR_INVALID_ARG, "IPC handle of the wrong size")
+    out = C.c_void_p()
+    check(None, lib.h3dit_ipc_open(handle, offset, C.byref(out)))
+    return int(out.value)
+
+
+def ipc_close(ptr: int, offset: int) -> None:
+    check(None, lib.h3dit_ipc_close(ptr, offset))
 
 
 class Context:
@@ -343,11 +373,12 @@ class Context:
                                         _stream(stream)))
 
     def empty(self, shape, kind: str):
-        """A device buffer for the sequence-parallel driver: "act" is bf16
-        (token-major activations), "f32" and "rope" are fp32."""
+        """A device buffer for the sequence-parallel driver: "act" and
+        "exchange" (activations other ranks write into) are bf16, "f32" and
+        "rope" are fp32."""
         import torch
 
-        dt = torch.bfloat16 if kind == "act" else torch.float32
+        dt = torch.bfloat16 if kind in ("act", "exchange") else torch.float32
         return torch.empty(*shape, dtype=dt, device="cuda")
 
     def attention_heads(self, heads: int, q, k, v, ld_qkv: int, o, ld_o: int, n: int,
@@ -365,6 +396,28 @@ class Context:
         """recv [ranks][n_local][I/ranks] -> o [n_local, I]."""
         self._check(lib.h3dit_sp_unpack_o(self.handle, _ptr(recv), o.shape[0], ranks, _ptr(o),
                                           _stream(stream)))
+
+    def sp_qkv_scatter(self, xm, w_qkv, rope_rows, recv_ptrs: Sequence[int], rank: int,
+                       stream=None) -> None:
+        """QKV + RoPE on this rank's rows xm [n_local, D], each head group's
+        Q|K|V stored straight into rank g's receive buffer at device address
+        recv_ptrs[g] (bf16 [ranks * n_local, 3I/ranks]): the first Ulysses
+        all-to-all fused into the GEMM's epilogue."""
+        arr = (C.c_void_p * len(recv_ptrs))(*recv_ptrs)
+        self._check(lib.h3dit_sp_qkv_scatter(self.handle, _ptr(xm), xm.shape[0], _ptr(w_qkv),
+                                             _ptr(rope_rows), arr, len(recv_ptrs), rank,
+                                             _stream(stream)))
+
+    def sp_attention_scatter(self, qkv_recv, o_ptrs: Sequence[int], rank: int,
+                             stream=None) -> None:
+        """Attention of this rank's head group over all tokens of qkv_recv
+        [N, 3I/ranks], each output row stored straight into the out-projection
+        input of the rank that holds it (device address o_ptrs[r], bf16
+        [N / ranks, I]): the second all-to-all fused into the epilogue."""
+        arr = (C.c_void_p * len(o_ptrs))(*o_ptrs)
+        self._check(lib.h3dit_sp_attention_scatter(self.handle, _ptr(qkv_recv),
+                                                   qkv_recv.shape[0], arr, len(o_ptrs), rank,
+                                                   _stream(stream)))
 
     def block_forward(self, block: int, t: float, x_img, grids, x_txt, mod=None,
                       stream=None) -> None:

@@ -20,9 +20,19 @@ module holds the buffers, slices the sequence and calls the collective it is
 given - torch.distributed.all_to_all_single (NCCL) between GPUs. Nothing here
 computes any of the method's arithmetic.
 
+The fused form (FusedUlyssesRank, fused_block) does the same exchanges with
+no collective and no re-layout kernel: the QKV GEMM's epilogue stores each
+head group's Q|K|V straight into the receive buffer of the rank that attends
+over it, and the attention's epilogue stores each output row straight into
+the out-projection input of the rank that holds the token
+(h3dit_sp_qkv_scatter / h3dit_sp_attention_scatter). Between GPUs the
+buffers are peer memory mapped with CUDA IPC (connect_peers), and a barrier
+after each of the two stages orders the writes against the reads.
+
 `ops` is the binding's Context, or any object with the same methods and an
 `empty(shape, kind)` allocator (kind "act" for the token-major activations,
-"f32" for fp32 vectors, "rope" for the RoPE table); the tests use an oracle-
+"exchange" for activations other ranks write into, "f32" for fp32 vectors,
+"rope" for the RoPE table); the tests use an oracle-
 backed one on the CPU to check the partition with real gloo ranks.
 """
 from __future__ import annotations
@@ -102,6 +112,142 @@ def block(rank: UlyssesRank, x, mod, w, rope_rows, all_to_all: Callable) -> None
     rank.finish(x, mod, w)
 
 
+class FusedUlyssesRank:
+    """One rank's buffers for the fused exchanges: `recv` [N, 3I/P] receives
+    the Q|K|V of this rank's heads from every rank's QKV GEMM, and `o`
+    [N/P, I] receives this rank's token rows of the attention output from
+    every rank's attention. `connect` takes every rank's `recv` and `o`
+    device addresses in rank order (its own included)."""
+
+    def __init__(self, ops, rank: int, world: int, n_total: int, hidden: int, heads: int,
+                 head_dim: int, ffn: int, max_ranks: int = 8):
+        if not 1 <= world <= max_ranks:
+            raise ValueError(f"the fused exchange addresses 1 .. {max_ranks} ranks, not {world}")
+        if n_total % world:
+            raise ValueError(f"{world} ranks do not divide {n_total} tokens")
+        if heads % world:
+            raise ValueError(f"{world} ranks do not divide {heads} heads")
+        self.ops, self.rank, self.world = ops, rank, world
+        self.n_total, self.n = n_total, n_total // world
+        self.D, self.H, self.dh, self.F = hidden, heads, head_dim, ffn
+        self.I = heads * head_dim
+        self.cw = self.I // world
+        e = ops.empty
+        self.xm = e((self.n, hidden), "act")
+        self.recv = e((n_total, 3 * self.cw), "exchange")  # written by every rank
+        self.o = e((self.n, self.I), "exchange")            # written by every rank
+        self.u = e((self.n, ffn), "act")
+        self.recv_ptrs: list | None = None
+        self.o_ptrs: list | None = None
+
+    def rows(self):
+        return slice(self.rank * self.n, (self.rank + 1) * self.n)
+
+    def connect(self, recv_ptrs: Sequence[int], o_ptrs: Sequence[int]) -> None:
+        if len(recv_ptrs) != self.world or len(o_ptrs) != self.world:
+            raise ValueError("one receive and one output address per rank")
+        self.recv_ptrs, self.o_ptrs = list(recv_ptrs), list(o_ptrs)
+
+    def qkv_scatter(self, x, mod, w, rope_rows) -> None:
+        """RMSNorm + modulate, then QKV + RoPE with the first exchange fused
+        in: every rank's `recv` gets this rank's rows of its head group."""
+        self.ops.rmsnorm_modulate(x, mod[0], mod[1], self.xm)
+        self.ops.sp_qkv_scatter(self.xm, w["w_qkv"], rope_rows, self.recv_ptrs, self.rank)
+
+    def attention_scatter(self) -> None:
+        """Attention of this rank's heads over all tokens, with the second
+        exchange fused in: every rank's `o` gets its rows for these heads."""
+        self.ops.sp_attention_scatter(self.recv, self.o_ptrs, self.rank)
+
+    def finish(self, x, mod, w) -> None:
+        ops = self.ops
+        ops.linear(H3DIT_EPI_GATED_RESIDUAL, self.o, w["w_o"], x, gate=mod[2])
+        ops.rmsnorm_modulate(x, mod[3], mod[4], self.xm)
+        ops.linear(H3DIT_EPI_GELU, self.xm, w["w_ff1"], self.u)
+        ops.linear(H3DIT_EPI_GATED_RESIDUAL, self.u, w["w_ff2"], x, gate=mod[5])
+
+
+def fused_block(rank: FusedUlyssesRank, x, mod, w, rope_rows, barrier: Callable) -> None:
+    """One block with the fused exchanges. barrier() must return only when
+    every rank's work so far has completed on its GPU: after the first stage
+    the attention reads what all ranks wrote, and after the second the
+    out-projection does; the next block's first stage then overwrites `recv`,
+    which every rank has finished reading by the second barrier."""
+    rank.qkv_scatter(x, mod, w, rope_rows)
+    barrier()
+    rank.attention_scatter()
+    barrier()
+    rank.finish(x, mod, w)
+
+
+def connect_peers(rank: FusedUlyssesRank, ipc=None, group=None) -> list:
+    """Maps every other rank's `recv` and `o` into this process and connects
+    the rank. The (handle, offset) pairs naming each rank's buffers are
+    exchanged with all_gather_object; an allocation is opened once even when
+    both buffers sit in it. `ipc` supplies handle(t) -> (bytes, offset),
+    open(handle) -> base address and close(base) (the binding's CUDA IPC by
+    default). Returns the opened base addresses, for close_peers."""
+    import torch.distributed as dist
+
+    if ipc is None:
+        from . import h3dit as H
+
+        ipc = _BindingIpc(H)
+    mine = (ipc.handle(rank.recv), ipc.handle(rank.o))
+    everyone = [None] * rank.world
+    dist.all_gather_object(everyone, mine, group=group)
+    bases: dict = {}
+    recv_ptrs, o_ptrs = [], []
+    for r, ((h_recv, off_recv), (h_o, off_o)) in enumerate(everyone):
+        if r == rank.rank:
+            recv_ptrs.append(rank.recv.data_ptr())
+            o_ptrs.append(rank.o.data_ptr())
+            continue
+        for h in (h_recv, h_o):
+            if h not in bases:
+                bases[h] = ipc.open(h)
+        recv_ptrs.append(bases[h_recv] + off_recv)
+        o_ptrs.append(bases[h_o] + off_o)
+    rank.connect(recv_ptrs, o_ptrs)
+    return list(bases.values())
+
+
+def close_peers(bases: Sequence[int], ipc=None) -> None:
+    if ipc is None:
+        from . import h3dit as H
+
+        ipc = _BindingIpc(H)
+    for b in bases:
+        ipc.close(b)
+
+
+class _BindingIpc:
+    def __init__(self, H):
+        self.H = H
+
+    def handle(self, t):
+        return self.H.ipc_handle(t)
+
+    def open(self, h):
+        return self.H.ipc_open(h, 0)
+
+    def close(self, base):
+        self.H.ipc_close(base, 0)
+
+
+def host_barrier(group=None) -> Callable:
+    """The barrier fused_block needs between GPUs: this rank's stream
+    drained, then a barrier across the ranks."""
+    import torch
+    import torch.distributed as dist
+
+    def barrier():
+        torch.cuda.current_stream().synchronize()
+        dist.barrier(group=group)
+
+    return barrier
+
+
 class UlyssesStep:
     """A sampling step under Ulysses SP on this rank: the timestep MLP, every
     block's AdaLN projection and the sequence's RoPE table are computed on
@@ -109,8 +255,17 @@ class UlyssesStep:
 
     def __init__(self, ops, weights: Sequence[dict], rank: int, world: int, n_total: int,
                  hidden: int, heads: int, head_dim: int, ffn: int,
-                 all_to_all: Callable | None = None, group=None):
-        self.r = UlyssesRank(ops, rank, world, n_total, hidden, heads, head_dim, ffn)
+                 all_to_all: Callable | None = None, group=None, fused: bool = False,
+                 barrier: Callable | None = None, ipc=None):
+        self.fused = fused
+        self.peer_bases: list = []
+        if fused:
+            # collective: every rank constructs its step at the same point
+            self.r = FusedUlyssesRank(ops, rank, world, n_total, hidden, heads, head_dim, ffn)
+            self.peer_bases = connect_peers(self.r, ipc=ipc, group=group)
+            self.barrier = barrier if barrier is not None else host_barrier(group)
+        else:
+            self.r = UlyssesRank(ops, rank, world, n_total, hidden, heads, head_dim, ffn)
         self.ops, self.weights = ops, list(weights)
         self.c = ops.empty((hidden,), "f32")
         self.mod = ops.empty((len(self.weights), 6, hidden), "f32")
@@ -129,4 +284,13 @@ class UlyssesStep:
         ops.rope_table(grids, n_txt, self.rope)
         rope_rows = self.rope[self.r.rows()]
         for l, w in enumerate(self.weights):
-            block(self.r, x, self.mod[l], w, rope_rows, self.all_to_all)
+            if self.fused:
+                fused_block(self.r, x, self.mod[l], w, rope_rows, self.barrier)
+            else:
+                block(self.r, x, self.mod[l], w, rope_rows, self.all_to_all)
+
+    def close(self, ipc=None) -> None:
+        """Unmaps the peers' buffers (fused form): call on every rank after
+        the last step, once every rank has stopped writing."""
+        close_peers(self.peer_bases, ipc)
+        self.peer_bases = []

@@ -266,6 +266,61 @@ h3dit_status h3dit_sp_pack_qkv(h3dit_ctx *ctx, const void *qkv, int32_t n_local,
 h3dit_status h3dit_sp_unpack_o(h3dit_ctx *ctx, const void *recv, int32_t n_local, int32_t ranks,
                                void *o, void *cuda_stream);
 
+/* The same two exchanges fused into the kernels that produce the data, for
+ * ranks whose buffers are mapped into one another's address space (peer
+ * memory over NVLink, opened with h3dit_ipc_open; or, on one GPU, plain
+ * device buffers of emulated ranks). No NCCL call and no re-layout kernel:
+ * the producing kernel stores each 16-byte piece straight into the rank that
+ * needs it. ranks: 1 .. H3DIT_MAX_SCATTER_RANKS, dividing cfg->heads, with
+ * heads*head_dim/ranks a multiple of 8; every pointer 16-byte aligned.
+ * The calls do not synchronise between ranks: before a rank reads what the
+ * others wrote (the attention after the QKV call, the out-projection after the
+ * attention call), every rank's call must have completed, and before a rank
+ * writes into a buffer, its owner must be done reading the previous
+ * contents. The caller provides this with a barrier after each call (a
+ * stream synchronise and a host barrier across the ranks); on one GPU, stream
+ * order provides it. Errors: H3DIT_ERR_INVALID_ARG for NULL or misaligned
+ * pointers, rank outside [0, ranks) or a bad count; H3DIT_ERR_UNSUPPORTED for
+ * ranks that do not divide the heads, more than H3DIT_MAX_SCATTER_RANKS ranks,
+ * or n_total not a multiple of ranks. */
+#define H3DIT_MAX_SCATTER_RANKS 8
+
+/* a4 with the first all-to-all: RMS-normalised, modulated tokens xm (device
+ * bf16 [n_local, D], this rank's rows `rank` * n_local ..) times w_qkv, RoPE
+ * on Q and K with rope_rows (this rank's rows of the sequence's table), each
+ * head group's Q | K | V columns stored into recv[g] (device bf16
+ * [ranks * n_local, 3I/ranks], rank g's receive buffer; recv is a host array
+ * of `ranks` pointers) at rows rank*n_local .. - the layout that
+ * h3dit_sp_pack_qkv plus the all-to-all produce. */
+h3dit_status h3dit_sp_qkv_scatter(h3dit_ctx *ctx, const void *xm, int32_t n_local,
+                                  const void *w_qkv, const float *rope_rows, void *const *recv,
+                                  int32_t ranks, int32_t rank, void *cuda_stream);
+
+/* a5 with the second all-to-all: attention of this rank's head group (heads
+ * rank*H/ranks ..) over all n_total tokens, reading qkv (device bf16
+ * [n_total, 3I/ranks], this rank's receive buffer), each output row t stored
+ * into o[t / n_local] (device bf16 [n_local, I], the out-projection input of
+ * the rank that holds token t; o is a host array of `ranks` pointers) at row
+ * t % n_local, columns rank*I/ranks .. (rank+1)*I/ranks - 1. */
+h3dit_status h3dit_sp_attention_scatter(h3dit_ctx *ctx, const void *qkv, int32_t n_total,
+                                        void *const *o, int32_t ranks, int32_t rank,
+                                        void *cuda_stream);
+
+/* Peer-memory mapping for the calls above (CUDA IPC; host calls, no kernel).
+ * h3dit_ipc_get_handle writes H3DIT_IPC_HANDLE_BYTES bytes that name the
+ * allocation holding the device pointer dev_ptr, and *offset_out, dev_ptr's
+ * byte offset in it; another process on the same node opens them with
+ * h3dit_ipc_open, which maps the allocation (peer access enabled on demand)
+ * and returns the address of the same byte in *dev_ptr_out. h3dit_ipc_close
+ * unmaps what h3dit_ipc_open returned (pass that pointer, offset included).
+ * Errors: H3DIT_ERR_INVALID_ARG for NULL arguments, H3DIT_ERR_CUDA when the
+ * runtime refuses (the handle is from this process, the peer is not
+ * reachable). */
+#define H3DIT_IPC_HANDLE_BYTES 64
+h3dit_status h3dit_ipc_get_handle(const void *dev_ptr, void *handle_out, uint64_t *offset_out);
+h3dit_status h3dit_ipc_open(const void *handle, uint64_t offset, void **dev_ptr_out);
+h3dit_status h3dit_ipc_close(void *dev_ptr, uint64_t offset);
+
 /* ---- a11: the MXFP8 variant of the four block linears ------------------
  * "H3-Image Day-0 Support: 4K in 0.87s with Vera Rubin", "Faster DiT" and
  * "Rubin Bringup": MXFP8 GEMMs for the eligible DiT linears. Format (a

@@ -139,8 +139,27 @@ def test_null_context_is_rejected_everywhere():
     io = H.h3dit_io_weights(0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 0x10000)
     assert H.lib.h3dit_denoise(None, C.byref(io), 0x10000, 24, 4, 4, 0x10000, 8, 6, None) \
         == H.H3DIT_ERR_INVALID_ARG
+    dst = (C.c_void_p * 2)(0x10000, 0x20000)
+    assert H.lib.h3dit_sp_qkv_scatter(None, 0x10000, 4, 0x10000, 0x10000, dst, 2, 0, None) \
+        == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_sp_attention_scatter(None, 0x10000, 8, dst, 2, 0, None) \
+        == H.H3DIT_ERR_INVALID_ARG
     H.lib.h3dit_destroy(None)  # NULL-safe
     assert H.lib.h3dit_last_error(None) == b"no context"
+
+
+def test_ipc_calls_reject_null_arguments_before_the_runtime():
+    off = C.c_uint64()
+    ptr = C.c_void_p()
+    handle = bytes(H.H3DIT_IPC_HANDLE_BYTES)
+    assert H.lib.h3dit_ipc_get_handle(None, handle, C.byref(off)) == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_ipc_get_handle(0x10000, None, C.byref(off)) == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_ipc_get_handle(0x10000, handle, None) == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_ipc_open(None, 0, C.byref(ptr)) == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_ipc_open(handle, 0, None) == H.H3DIT_ERR_INVALID_ARG
+    assert H.lib.h3dit_ipc_close(None, 0) == H.H3DIT_ERR_INVALID_ARG
+    with pytest.raises(H.H3DitError):
+        H.ipc_open(b"short", 0)  # the binding checks the handle's size
 
 
 def test_mx_scale_layout_size():

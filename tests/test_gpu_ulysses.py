@@ -99,6 +99,140 @@ def test_emulated_ranks_full_width_4096(P):
     assert torch.equal(got, ref), f"max diff {float((got - ref).abs().max())}"
 
 
+def _emulated_step_fused(ctx, weights, P, dims, t, x, grids, n_txt):
+    """The fused form: each rank's QKV GEMM and attention write straight into
+    the other ranks' buffers (here all on one GPU, so stream order stands in
+    for the barrier between the stages)."""
+    from image_generation_b200.ulysses import FusedUlyssesRank, fused_block
+
+    n_total = x.shape[0]
+    ranks = [FusedUlyssesRank(ctx, r, P, n_total, dims.hidden, dims.heads, dims.head_dim,
+                              dims.ffn) for r in range(P)]
+    recv_ptrs = [r.recv.data_ptr() for r in ranks]
+    o_ptrs = [r.o.data_ptr() for r in ranks]
+    for r in ranks:
+        r.recv.fill_(float("nan"))
+        r.o.fill_(float("nan"))
+        r.connect(recv_ptrs, o_ptrs)
+    c = torch.empty(dims.hidden, device="cuda")
+    mod = torch.empty(len(weights), 6, dims.hidden, device="cuda")
+    rope = torch.empty(n_total, dims.head_dim // 2, 2, device="cuda")
+    ctx.time_embed(t, c)
+    ctx.adaln_project(c, 0, len(weights), mod)
+    ctx.rope_table(grids, n_txt, rope)
+    xs = [x[r.rows()].clone() for r in ranks]
+    for l, w in enumerate(weights):
+        for i, r in enumerate(ranks):
+            r.qkv_scatter(xs[i], mod[l], w, rope[r.rows()])
+        for r in ranks:
+            r.attention_scatter()
+        for i, r in enumerate(ranks):
+            r.finish(xs[i], mod[l], w)
+    return torch.cat(xs)
+
+
+def _run_fused(dims, n_blocks, P, n_txt, grids, seed):
+    from image_generation_b200 import h3dit as H
+
+    tw = time_tensors(synth.time_weights(dims, seed))
+    weights = [block_tensors(synth.block_weights(dims, seed + 100 + l)) for l in range(n_blocks)]
+    n_total = n_txt + sum(h * w for _, h, w in grids)
+    cfg = H.make_config(dims.hidden, dims.heads, dims.head_dim, dims.ffn, n_blocks, n_total,
+                        io_fp32=True)
+    ctx = H.Context(cfg, tw, weights)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    x = torch.randn(n_total, dims.hidden, device="cuda", generator=g)
+    got = _emulated_step_fused(ctx, weights, P, dims, 0.4, x, grids, n_txt)
+    xt, xi = x[:n_txt].clone(), x[n_txt:].clone()
+    ctx.step(0.4, xi, grids, xt)
+    torch.cuda.synchronize()
+    assert ctx.sync_status() == 0
+    ref = torch.cat([xt, xi])
+    assert not torch.equal(ref, x)
+    return got, ref
+
+
+@pytest.mark.parametrize("P", [1, 2, 4, 8])
+def test_fused_exchange_emulated_ranks_small(P):
+    got, ref = _run_fused(synth.SMALL, 2, P, 32, [(0, 16, 16)], 1)
+    assert torch.equal(got, ref), f"max diff {float((got - ref).abs().max())}"
+
+
+def test_fused_exchange_head_dim_128_ragged_tiles():
+    """d_h 128 (rotary units of 32 and 48 columns) on 4 x 300 = 1,200 tokens:
+    each rank's 300 rows end inside a 256-row GEMM tile, and the attention's
+    last query and key tiles run past the sequence."""
+    dims = synth.Dims(hidden=768, heads=8, head_dim=128, ffn=2048)
+    got, ref = _run_fused(dims, 2, 4, 8, [(0, 32, 37), (1, 4, 2)], 2)
+    assert torch.equal(got, ref), f"max diff {float((got - ref).abs().max())}"
+
+
+@pytest.mark.parametrize("P", [4, 8])
+def test_fused_exchange_full_width_4096(P):
+    """SP4 and SP8 at full width on the 4096^2 sequence, one block."""
+    got, ref = _run_fused(synth.FULL_96, 1, P, 512, [(0, 128, 128)], 3)
+    assert torch.equal(got, ref), f"max diff {float((got - ref).abs().max())}"
+
+
+def test_fused_exchange_writes_only_its_blocks():
+    """Every receive and output buffer sits between guard margins; the two
+    fused calls of all ranks must fill the buffers and leave the margins."""
+    from image_generation_b200 import h3dit as H
+    from tests.test_gpu_guards import Guarded
+
+    dims, P, n_txt, grids = synth.SMALL, 4, 4, [(0, 10, 10)]
+    n_total = n_txt + 100
+    n = n_total // P
+    cw = dims.inner // P
+    cfg = H.make_config(dims.hidden, dims.heads, dims.head_dim, dims.ffn, 1, n_total)
+    bw = block_tensors(synth.block_weights(dims, 5))
+    ctx = H.Context(cfg, time_tensors(synth.time_weights(dims, 5)), [bw])
+    recv = [Guarded((n_total, 3 * cw), torch.bfloat16) for _ in range(P)]
+    outs = [Guarded((n, dims.inner), torch.bfloat16) for _ in range(P)]
+    rope = torch.empty(n_total, dims.head_dim // 2, 2, device="cuda")
+    ctx.rope_table(grids, n_txt, rope)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    xm = (torch.randn(n_total, dims.hidden, device="cuda", generator=g)).bfloat16()
+    for r in range(P):
+        ctx.sp_qkv_scatter(xm[r * n:(r + 1) * n], bw["w_qkv"], rope[r * n:(r + 1) * n],
+                           [b.t.data_ptr() for b in recv], r)
+    for r in range(P):
+        ctx.sp_attention_scatter(recv[r].t, [b.t.data_ptr() for b in outs], r)
+    torch.cuda.synchronize()
+    assert ctx.sync_status() == 0
+    for i, b in enumerate(recv + outs):
+        b.check(f"buffer {i}")
+        assert not bool(torch.isnan(b.t.float()).any())
+
+
+def test_fused_exchange_errors():
+    from image_generation_b200 import h3dit as H
+
+    dims = synth.SMALL
+    cfg = H.make_config(dims.hidden, dims.heads, dims.head_dim, dims.ffn, 1, 64)
+    bw = block_tensors(synth.block_weights(dims, 0))
+    ctx = H.Context(cfg, time_tensors(synth.time_weights(dims, 0)), [bw])
+    xm = torch.zeros(16, dims.hidden, device="cuda", dtype=torch.bfloat16)
+    rope = torch.zeros(16, dims.head_dim // 2, 2, device="cuda")
+    buf = torch.zeros(64, 3 * dims.inner, device="cuda", dtype=torch.bfloat16)
+    p = buf.data_ptr()
+    cases = [
+        (lambda: ctx.sp_qkv_scatter(xm, bw["w_qkv"], rope, [p, p, p], 0), H.H3DIT_ERR_UNSUPPORTED),
+        (lambda: ctx.sp_qkv_scatter(xm, bw["w_qkv"], rope, [p] * 16, 0), H.H3DIT_ERR_UNSUPPORTED),
+        (lambda: ctx.sp_qkv_scatter(xm, bw["w_qkv"], rope, [p, p], 2), H.H3DIT_ERR_INVALID_ARG),
+        (lambda: ctx.sp_qkv_scatter(xm, bw["w_qkv"], rope, [p, p + 2], 0), H.H3DIT_ERR_INVALID_ARG),
+        (lambda: ctx.sp_qkv_scatter(xm, bw["w_qkv"], rope, [p, 0], 0), H.H3DIT_ERR_INVALID_ARG),
+        (lambda: ctx.sp_attention_scatter(buf[:63], [p, p], 0), H.H3DIT_ERR_UNSUPPORTED),
+    ]
+    for call, status in cases:
+        with pytest.raises(H.H3DitError) as e:
+            call()
+        assert e.value.status == status
+    assert ctx.sync_status() == 0
+
+
 def test_relayout_errors():
     from image_generation_b200 import h3dit as H
 

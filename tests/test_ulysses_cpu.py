@@ -187,3 +187,147 @@ def test_partition_rules():
         UlyssesRank(ops, 0, 5, 288, 768, 10, 96, 2048)  # 288 tokens over 5 ranks
     r = UlyssesRank(ops, 2, 4, 288, 768, 8, 96, 2048)
     assert r.rows() == slice(144, 216) and r.cw == 192
+
+
+# ---------------------------------------------------------------- fused form
+# The fused exchanges (h3dit_sp_qkv_scatter / h3dit_sp_attention_scatter)
+# write into other ranks' buffers. Here the ranks are gloo processes whose
+# exchange buffers live in one shared-memory arena, the CPU stand-in for
+# peer memory: a rank's "IPC handle" names the arena and a byte offset, and
+# the oracle ops below store into the addresses they are given, with the
+# layouts include/h3dit.h documents for the two calls.
+
+class ArenaIpc:
+    def __init__(self, arena):
+        self.arena, self.opened = arena, 0
+
+    def handle(self, t):
+        return b"arena", t.data_ptr() - self.arena.data_ptr()
+
+    def open(self, h):
+        assert h == b"arena"
+        self.opened += 1
+        return self.arena.data_ptr()
+
+    def close(self, base):
+        assert base == self.arena.data_ptr()
+
+
+class ArenaOracleOps(OracleOps):
+    """OracleOps whose "exchange" buffers are carved from the shared arena
+    (rank r's at its own offsets) and whose fused-exchange calls write to
+    arena addresses."""
+
+    def __init__(self, cfg, tw, bws, arena, rank, per_rank):
+        super().__init__(cfg, tw, bws)
+        self.arena, self.next = arena, rank * per_rank
+
+    def empty(self, shape, kind):
+        if kind != "exchange":
+            return super().empty(shape, kind)
+        size = int(np.prod(shape))
+        v = self.arena[self.next:self.next + size].view(*shape)
+        self.next += size
+        return v
+
+    def _at(self, ptr, shape):
+        off = ptr - self.arena.data_ptr()
+        assert off % 8 == 0 and off >= 0
+        i = off // 8
+        return self.arena[i:i + int(np.prod(shape))].view(*shape)
+
+    def sp_qkv_scatter(self, xm, w_qkv, rope_rows, recv_ptrs, rank):
+        n, I, P = xm.shape[0], self.cfg.inner, len(recv_ptrs)
+        cw = I // P
+        y = torch.empty(n, 3 * I, dtype=torch.float64)
+        self.linear(EPI_QKV_ROPE, xm, w_qkv, y, rope_table=rope_rows)
+        for g, ptr in enumerate(recv_ptrs):
+            dst = self._at(ptr, (P * n, 3 * cw))
+            for m in range(3):
+                dst[rank * n:(rank + 1) * n, m * cw:(m + 1) * cw] = \
+                    y[:, m * I + g * cw:m * I + (g + 1) * cw]
+
+    def sp_attention_scatter(self, recv, o_ptrs, rank):
+        n_all, P = recv.shape[0], len(o_ptrs)
+        cw, n = self.cfg.inner // P, recv.shape[0] // len(o_ptrs)
+        o_heads = torch.empty(n_all, cw, dtype=torch.float64)
+        self.attention_heads(self.cfg.heads // P, recv[:, :cw], recv[:, cw:2 * cw],
+                             recv[:, 2 * cw:], 3 * cw, o_heads, cw, n_all)
+        for p, ptr in enumerate(o_ptrs):
+            dst = self._at(ptr, (n, self.cfg.inner))
+            dst[:, rank * cw:(rank + 1) * cw] = o_heads[p * n:(p + 1) * n]
+
+
+def _fused_sizes(dims, n_total, world):
+    cw = dims.heads * dims.head_dim // world
+    return n_total * 3 * cw + (n_total // world) * dims.heads * dims.head_dim
+
+
+def _fused_rank_main(rank, world, port, head_dim, arena, out):
+    import torch.distributed as dist
+
+    from image_generation_b200.ulysses import UlyssesStep
+
+    torch.set_num_threads(2)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        dims, cfg, tw, bws, n_txt, grids, x = _case(head_dim)
+        n_total = x.shape[0]
+        ops = ArenaOracleOps(cfg, tw, bws, arena, rank, _fused_sizes(dims, n_total, world))
+        ipc = ArenaIpc(arena)
+        step = UlyssesStep(ops, [dict(b) for b in bws], rank, world, n_total, dims.hidden,
+                           dims.heads, dims.head_dim, dims.ffn, fused=True,
+                           barrier=dist.barrier, ipc=ipc)
+        assert ipc.opened == (1 if world > 1 else 0)  # one arena, opened once
+        assert step.r.recv_ptrs[rank] == step.r.recv.data_ptr()
+        xl = torch.from_numpy(x[step.r.rows()].copy())
+        step(0.6, xl, grids, n_txt)
+        dist.barrier()
+        step.close(ipc)
+        rows = [torch.empty_like(xl) for _ in range(world)]
+        dist.all_gather(rows, xl)
+        if rank == 0:
+            out["y"] = torch.cat(rows).numpy()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,head_dim", [(2, 96), (4, 96), (2, 128)],
+                         ids=["sp2", "sp4", "sp2_dh128"])
+def test_fused_exchange_ranks_match_the_unsharded_step(world, head_dim):
+    """The fused form: no all-to-all and no re-layout; each rank's QKV and
+    attention write straight into the other ranks' buffers (here a shared
+    arena), ordered by a barrier after each stage."""
+    dims, cfg, tw, bws, n_txt, grids, x = _case(head_dim)
+    arena = torch.full((world * _fused_sizes(dims, x.shape[0], world),), float("nan"),
+                       dtype=torch.float64).share_memory_()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_fused_rank_main, args=(r, world, port, head_dim, arena, out))
+                 for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=300)
+        assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+        y = out["y"]
+    ref = O.step_forward(x, 0.6, tw, bws, O.token_positions(n_txt, grids), cfg)
+    assert np.abs(y - ref).max() <= 1e-12 * np.abs(ref).max()
+    assert np.abs(y - x).max() > 1e-3
+
+
+def test_fused_partition_rules():
+    from image_generation_b200.ulysses import FusedUlyssesRank
+
+    ops = OracleOps(None, None, None)
+    with pytest.raises(ValueError):
+        FusedUlyssesRank(ops, 0, 16, 288, 768, 16, 96, 2048)  # more ranks than addressable
+    with pytest.raises(ValueError):
+        FusedUlyssesRank(ops, 0, 3, 288, 768, 8, 96, 2048)    # 3 ranks, 8 heads
+    r = FusedUlyssesRank(ops, 1, 4, 288, 768, 8, 96, 2048)
+    assert tuple(r.recv.shape) == (288, 3 * 192) and tuple(r.o.shape) == (72, 768)
+    with pytest.raises(ValueError):
+        r.connect([0, 1, 2], [0, 1, 2, 3])
