@@ -193,21 +193,28 @@ def connect_peers(rank: FusedUlyssesRank, ipc=None, group=None) -> list:
         from . import h3dit as H
 
         ipc = _BindingIpc(H)
-    mine = (ipc.handle(rank.recv), ipc.handle(rank.o))
+    def named(t):
+        h, off = ipc.handle(t)
+        return h, off, t.data_ptr() - off  # the allocation's base in the owner
+
+    mine = (named(rank.recv), named(rank.o))
     everyone = [None] * rank.world
     dist.all_gather_object(everyone, mine, group=group)
     bases: dict = {}
     recv_ptrs, o_ptrs = [], []
-    for r, ((h_recv, off_recv), (h_o, off_o)) in enumerate(everyone):
+    for r, pair in enumerate(everyone):
         if r == rank.rank:
             recv_ptrs.append(rank.recv.data_ptr())
             o_ptrs.append(rank.o.data_ptr())
             continue
-        for h in (h_recv, h_o):
-            if h not in bases:
-                bases[h] = ipc.open(h)
-        recv_ptrs.append(bases[h_recv] + off_recv)
-        o_ptrs.append(bases[h_o] + off_o)
+        ptrs = []
+        for h, off, owner_base in pair:
+            key = (r, owner_base)  # one opening per allocation of each rank
+            if key not in bases:
+                bases[key] = ipc.open(h)
+            ptrs.append(bases[key] + off)
+        recv_ptrs.append(ptrs[0])
+        o_ptrs.append(ptrs[1])
     rank.connect(recv_ptrs, o_ptrs)
     return list(bases.values())
 

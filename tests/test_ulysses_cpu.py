@@ -279,7 +279,9 @@ def _fused_rank_main(rank, world, port, head_dim, arena, out):
         step = UlyssesStep(ops, [dict(b) for b in bws], rank, world, n_total, dims.hidden,
                            dims.heads, dims.head_dim, dims.ffn, fused=True,
                            barrier=dist.barrier, ipc=ipc)
-        assert ipc.opened == (1 if world > 1 else 0)  # one arena, opened once
+        # each peer's two exchange buffers sit in one allocation (the arena),
+        # which is opened once per peer
+        assert ipc.opened == world - 1
         assert step.r.recv_ptrs[rank] == step.r.recv.data_ptr()
         xl = torch.from_numpy(x[step.r.rows()].copy())
         step(0.6, xl, grids, n_txt)
