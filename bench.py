@@ -61,6 +61,8 @@ def parse():
     ap.add_argument("--no-mxfp8", action="store_true")
     ap.add_argument("--no-vae", action="store_true",
                     help="skip the VAE decoder timing")
+    ap.add_argument("--no-sp", action="store_true",
+                    help="skip the one-GPU timing of a block under Ulysses SP4 (fused exchanges)")
     ap.add_argument("--no-streaming", action="store_true",
                     help="skip the layerwise weight-streaming timings")
     ap.add_argument("--no-denoise", action="store_true",
@@ -785,6 +787,76 @@ def denoise_timing(ctx, x_txt, rank, world, barrier, dist, stream, reps: int = 2
                     "h2d_bytes_per_run": in_bytes, "d2h_bytes_per_run": h_out.numel() * 4}}
 
 
+def sp_fused_timing(ctx, block, ranks: int = 4, reps: int = 3) -> dict:
+    """One block of the 4096^2 step under Ulysses SP with the fused exchanges,
+    all `ranks` ranks on this one GPU: each rank's three stages (RMSNorm +
+    QKV storing into every rank's receive buffer; attention of its head group
+    storing into every rank's out-projection input; out-projection and FFN)
+    through the library, timed per stage with CUDA events, next to the
+    unsharded block. On one GPU the ranks run one after another, so the total
+    is the block's whole work plus the decomposition's overhead; the per-rank
+    stage times are what one GPU of an SP group would spend."""
+    import torch
+
+    from image_generation_b200.ulysses import FusedUlyssesRank
+
+    n_total = N_TOK
+    rs = [FusedUlyssesRank(ctx, r, ranks, n_total, D, H, ctx.cfg.head_dim, F)
+          for r in range(ranks)]
+    for r in rs:
+        r.connect([q.recv.data_ptr() for q in rs], [q.o.data_ptr() for q in rs])
+    c = torch.empty(D, device="cuda")
+    mod = torch.empty(1, 6, D, device="cuda")
+    rope = torch.empty(n_total, ctx.cfg.head_dim // 2, 2, device="cuda")
+    ctx.time_embed(0.5, c)
+    ctx.adaln_project(c, 0, 1, mod)
+    ctx.rope_table([(0, GRID, GRID)], N_TXT, rope)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7)
+    x = torch.randn(n_total, D, device="cuda", generator=g)
+    xs = [x[r.rows()].clone() for r in rs]
+    stages = ("qkv_scatter", "attention_scatter", "finish")
+    ev = {s: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(ranks)] for s in stages}
+    times = {s: [] for s in stages}
+    for rep in range(reps + 1):
+        for i, r in enumerate(rs):
+            ev["qkv_scatter"][i][0].record()
+            r.qkv_scatter(xs[i], mod[0], block, rope[r.rows()])
+            ev["qkv_scatter"][i][1].record()
+        for i, r in enumerate(rs):
+            ev["attention_scatter"][i][0].record()
+            r.attention_scatter()
+            ev["attention_scatter"][i][1].record()
+        for i, r in enumerate(rs):
+            ev["finish"][i][0].record()
+            r.finish(xs[i], mod[0], block)
+            ev["finish"][i][1].record()
+        torch.cuda.synchronize()
+        if rep:  # the first pass warms up
+            for s in stages:
+                times[s].append(sum(a.elapsed_time(b) for a, b in ev[s]) / ranks)
+    if ctx.sync_status() != 0:
+        raise RuntimeError("sequence-parallel stages failed")
+    per_rank = {s: round(sorted(v)[len(v) // 2], 3) for s, v in times.items()}
+    xt = torch.randn(N_TXT, D, device="cuda", generator=g).bfloat16()
+    xi = torch.randn(GRID * GRID, D, device="cuda", generator=g).bfloat16()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ctx.block_forward(0, 0.5, xi, [(0, GRID, GRID)], xt, mod=mod[0])
+    e0.record()
+    for _ in range(reps):
+        ctx.block_forward(0, 0.5, xi, [(0, GRID, GRID)], xt, mod=mod[0])
+    e1.record()
+    torch.cuda.synchronize()
+    if ctx.sync_status() != 0:
+        raise RuntimeError("unsharded block failed")
+    return {"ranks": ranks, "tokens": n_total, "ms_per_rank": per_rank,
+            "ms_per_rank_total": round(sum(per_rank.values()), 3),
+            "ms_unsharded_block": round(e0.elapsed_time(e1) / reps, 3),
+            "note": "all ranks on one GPU, one after another; the exchanges are the QKV and "
+                    "attention epilogues' stores into the other ranks' buffers"}
+
+
 def optional_leg(name: str, fn):
     """Run one of the extra measurements; a failure there is reported in its
     field instead of costing the whole line (the step's own timing is not
@@ -924,6 +996,10 @@ def run_h3dit(args):
             streaming["resident_50"] = {"ms_per_step": round(ms_step, 1), "streamed_blocks": 0,
                                         "h2d_bytes_per_step": 0}
 
+    sp = None
+    if world == 1 and not args.no_sp and dh == 96:
+        sp = optional_leg("sp_fused", lambda: sp_fused_timing(ctx, blocks[0]))
+
     line = None
     if rank == 0:
         peaks, peak_src = load_peaks()
@@ -978,6 +1054,7 @@ def run_h3dit(args):
             "denoise_6step": denoise,
             "weight_streaming": streaming,
             "vae_decode_4096": vae,
+            "ulysses_sp4_fused_one_gpu": sp,
             "graph_ms_per_step": None if graph_ms is None else round(graph_ms, 2),
         }
         gemm_kinds = ("qkv", "out_proj", "ffn1", "ffn2")
