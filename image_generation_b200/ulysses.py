@@ -182,9 +182,10 @@ def fused_block(rank: FusedUlyssesRank, x, mod, w, rope_rows, barrier: Callable)
 
 def connect_peers(rank: FusedUlyssesRank, ipc=None, group=None) -> list:
     """Maps every other rank's `recv` and `o` into this process and connects
-    the rank. The (handle, offset) pairs naming each rank's buffers are
-    exchanged with all_gather_object; an allocation is opened once even when
-    both buffers sit in it. `ipc` supplies handle(t) -> (bytes, offset),
+    the rank. Each buffer is named by (handle, byte offset, the allocation's
+    base address in its owner); the names are exchanged with
+    all_gather_object, and an allocation is opened once even when both
+    buffers sit in it. `ipc` supplies handle(t) -> (bytes, offset),
     open(handle) -> base address and close(base) (the binding's CUDA IPC by
     default). Returns the opened base addresses, for close_peers."""
     import torch.distributed as dist
@@ -193,6 +194,7 @@ def connect_peers(rank: FusedUlyssesRank, ipc=None, group=None) -> list:
         from . import h3dit as H
 
         ipc = _BindingIpc(H)
+
     def named(t):
         h, off = ipc.handle(t)
         return h, off, t.data_ptr() - off  # the allocation's base in the owner
