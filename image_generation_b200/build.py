@@ -1,6 +1,7 @@
 """Build libh3dit.so in-tree with nvcc for sm_100a (no GPU needed to build).
 
-    python -m image_generation_b200.build [-v]
+    python -m image_generation_b200.build [-v]            # libh3dit.so
+    python -m image_generation_b200.build --stamps        # libh3dit_stamps.so (diagnostic)
 """
 from __future__ import annotations
 
@@ -58,5 +59,18 @@ def build(verbose: bool = False, extra=(), out: str = LIB, build_dir: str = BUIL
     return out
 
 
+LIB_STAMPS = os.path.join(PKG, "libh3dit_stamps.so")
+
+
+def build_stamps(verbose: bool = False) -> str:
+    """The diagnostic build: the product sources with the attention kernel's
+    clock-stamp points compiled in (read with h3dit_attention_stamps)."""
+    return build(verbose, extra=["-DH3_ATTN_STAMPS"], out=LIB_STAMPS,
+                 build_dir=BUILD + "_stamps")
+
+
 if __name__ == "__main__":
-    print(build(verbose="-v" in sys.argv))
+    if "--stamps" in sys.argv:
+        print(build_stamps(verbose="-v" in sys.argv))
+    else:
+        print(build(verbose="-v" in sys.argv))

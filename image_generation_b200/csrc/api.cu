@@ -1664,6 +1664,12 @@ h3dit_status h3dit_selftest_bounded_wait(h3dit_ctx *ctx, int32_t limit_us, void 
                    "self-test launch");
 }
 
+h3dit_status h3dit_attention_stamps(uint64_t *host, int32_t slots, int32_t steps) {
+  if (!host) return H3DIT_ERR_INVALID_ARG;
+  const int r = attention_stamps(reinterpret_cast<unsigned long long *>(host), slots, steps);
+  return r == 0 ? H3DIT_OK : r == 1 || r == -1 ? H3DIT_ERR_UNSUPPORTED : H3DIT_ERR_CUDA;
+}
+
 h3dit_status h3dit_profile_begin(h3dit_ctx *ctx) {
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
   ctx->recycle_records();

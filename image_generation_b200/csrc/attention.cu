@@ -36,6 +36,37 @@
 #include "ptx.cuh"
 
 namespace h3 {
+
+// Per-phase clock stamps of one CTA (the build with -DH3_ATTN_STAMPS only;
+// the product build compiles the stamp points away). Slot layout, one row of
+// kStampSlots per 64-key step j: softmax of query tile t (its first warp,
+// lane 0) at 6t + {S seen, scores loaded, row max, exponentials, P stored,
+// P handed back}; issuer of tile t at 12 + 3t + {P seen, PV issued, S(j+2)
+// issued}; TMA producer at 18 (stage free); hand-back of each softmax warp
+// of tile t at 20 + 4t + (warp % 4); issuer of tile t at 28 + t once K_j has
+// landed.
+constexpr int kStampSlots = 32, kStampSteps = 300;
+#ifdef H3_ATTN_STAMPS
+__device__ unsigned long long g_attn_stamps[kStampSlots * kStampSteps];
+#define H3_STAMP(on, j, slot)                                                      \
+  do {                                                                             \
+    if ((on) && (j) < kStampSteps) g_attn_stamps[(j) * kStampSlots + (slot)] = clock64(); \
+  } while (0)
+// the stamp may not move above the computation of `v`
+#define H3_STAMP_AFTER(on, j, slot, v)      \
+  do {                                      \
+    asm volatile("" ::"r"(__float_as_uint(v))); \
+    H3_STAMP(on, j, slot);                  \
+  } while (0)
+#else
+#define H3_STAMP(on, j, slot) \
+  do {                        \
+  } while (0)
+#define H3_STAMP_AFTER(on, j, slot, v) \
+  do {                                 \
+  } while (0)
+#endif
+
 namespace {
 
 constexpr int BQ = kAttnBQ;                  // rows of one query tile
@@ -163,6 +194,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   // stored, keys past n are masked below
   const int seq0 = blockIdx.z * p.n;
   const int nkv = p.tiles_kv;
+#ifdef H3_ATTN_STAMPS
+  const bool stamp_cta = blockIdx.x == 20 && blockIdx.y == 10 && blockIdx.z == 0;
+#endif
 
   if (threadIdx.x == 0) {
     mbar_init(Q_FULL, 1);
@@ -206,6 +240,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int j = 0; j < nkv; ++j) {
         const int st = j % NS;
         if (!mbar_wait(KV_EMPTY(st), ((j / NS) & 1) ^ 1, p.status)) break;
+        H3_STAMP(stamp_cta, j, 18);
         mbar_arrive_expect_tx(KV_FULL(st), 2 * DCH * KBOX);
         const uint32_t k_dst = sKV + st * STAGE_BYTES;
         const uint32_t v_dst = k_dst + KV_BYTES;
@@ -229,6 +264,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t q_tmem = tmem + QT_COL + 32 * t;
       auto issue_s = [&](int j) -> bool {
         if (!mbar_wait(KV_FULL(j % NS), (j / NS) & 1, p.status)) return false;
+        H3_STAMP(stamp_cta, j, 28 + t);
         tc_fence_after();
         const uint32_t k_src = sKV + (j % NS) * STAGE_BYTES;
 #pragma unroll
@@ -255,6 +291,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           ok = false;
           break;
         }
+        H3_STAMP(stamp_cta, j, 12 + 3 * t);
         tc_fence_after();
         const uint32_t v_src = sKV + (j % NS) * STAGE_BYTES + KV_BYTES;
 #pragma unroll
@@ -267,10 +304,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         umma_commit(PV_DONE(t));
         umma_commit(KV_EMPTY(j % NS));  // this tile no longer reads K_j, V_j
         if (j + 1 == nkv) umma_commit(O_FULL(t));
+        H3_STAMP(stamp_cta, j, 13 + 3 * t);
         if (j + SBUF < nkv && !issue_s(j + SBUF)) {
           ok = false;
           break;
         }
+        H3_STAMP(stamp_cta, j, 14 + 3 * t);
       }
       umma_commit(DRAIN(t));
       mbar_wait(DRAIN(t), 0, p.status, false);
@@ -314,6 +353,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         ok = false;
         break;
       }
+#ifdef H3_ATTN_STAMPS
+      const bool me = stamp_cta && sub == 0 && lane == 0;
+#endif
+      H3_STAMP(me, j, 6 * t + 0);
       tc_fence_after();
       const int valid = p.n - j * BKV;  // keys of this tile that exist
       float alpha = 1.f;
@@ -332,10 +375,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       {
         float sc[64];
         load_scores64(tS, sc, valid);
+        H3_STAMP_AFTER(me, j, 6 * t + 1, sc[63]);
         update_max(row_max64(sc));
+        H3_STAMP_AFTER(me, j, 6 * t + 2, m);
         uint32_t pk[32];
         exp_pack64(sc, sl2, m, part, pk);
+        H3_STAMP_AFTER(me, j, 6 * t + 3, __uint_as_float(pk[31]));
         tmem_st32(tS, pk);
+        H3_STAMP(me, j, 6 * t + 4);
       }
       float sum;
       {
@@ -364,6 +411,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(P_FULL(t, j % SBUF));
+      H3_STAMP(me, j, 6 * t + 5);
+      H3_STAMP(stamp_cta && lane == 0, j, 20 + 4 * t + sub);
     }
     if (ok) ok = mbar_wait(O_FULL(t), 0, p.status);
     if (__all_sync(0xffffffffu, ok)) {
@@ -440,6 +489,18 @@ cudaError_t launch_dh(const CUtensorMap &q, const CUtensorMap &k, const CUtensor
 }
 
 }  // namespace
+
+int attention_stamps(unsigned long long *host, int slots, int steps) {
+#ifdef H3_ATTN_STAMPS
+  if (slots != kStampSlots || steps != kStampSteps) return -1;
+  return cudaMemcpyFromSymbol(host, g_attn_stamps, sizeof(g_attn_stamps)) == cudaSuccess ? 0 : -2;
+#else
+  (void)host;
+  (void)slots;
+  (void)steps;
+  return 1;  // a build without the stamp points
+#endif
+}
 
 cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
                              const AttnParams &p, int head_dim, int heads, bool out_mx,

@@ -132,6 +132,10 @@ constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 64;
 
+// Copies the attention kernel's clock stamps (built with -DH3_ATTN_STAMPS)
+// to host: 0 on success, 1 in a build without them, negative on errors.
+int attention_stamps(unsigned long long *host, int slots, int steps);
+
 cudaError_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p,
                         int epilogue, int grid, cudaStream_t s);
 int gemm_smem_bytes();

@@ -13,7 +13,9 @@ import re
 from typing import List, Sequence, Tuple
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libh3dit.so")
+# H3DIT_LIB selects another build of the library (the stamped diagnostic
+# build); the product library is the default.
+LIB_PATH = os.environ.get("H3DIT_LIB") or os.path.join(PKG, "libh3dit.so")
 HEADER = os.path.join(os.path.dirname(PKG), "include", "h3dit.h")
 
 H3DIT_OK = 0
@@ -38,6 +40,8 @@ H3DIT_PRECISION_MXFP8 = 1
 H3DIT_STATIC_TIME_MAX_HIDDEN = 8192
 H3DIT_MAX_SCATTER_RANKS = 8
 H3DIT_IPC_HANDLE_BYTES = 64
+H3DIT_ATTN_STAMP_SLOTS = 32
+H3DIT_ATTN_STAMP_STEPS = 300
 
 KERNEL_KINDS = ["time_embed", "adaln", "rmsnorm", "qkv", "attention", "out_proj", "ffn1",
                 "ffn2", "rope_table", "pack", "mx_quantize", "io"]
@@ -151,6 +155,7 @@ def _load() -> C.CDLL:
         "h3dit_profile_begin": (i32, [p]),
         "h3dit_profile_end": (i32, [p, C.POINTER(C.c_float), C.POINTER(C.c_int64)]),
         "h3dit_launch_count": (C.c_int64, [p]),
+        "h3dit_attention_stamps": (i32, [C.POINTER(C.c_uint64), i32, i32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

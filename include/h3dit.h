@@ -618,6 +618,19 @@ h3dit_status h3dit_profile_end(h3dit_ctx *ctx, float *ms_out, int64_t *launches_
 /* Kernels this context has enqueued since it was created. */
 int64_t h3dit_launch_count(const h3dit_ctx *ctx);
 
+/* Per-phase clock stamps of the attention kernel, for the diagnostic build
+ * (`python -m image_generation_b200.build --stamps` writes
+ * libh3dit_stamps.so with the stamp points compiled in; the product library
+ * has none and returns H3DIT_ERR_UNSUPPORTED). One CTA of every launch (query
+ * tiles 40-41 of head 10) records clock64() at fixed points of each 64-key
+ * step into a device table of H3DIT_ATTN_STAMP_SLOTS x H3DIT_ATTN_STAMP_STEPS
+ * entries (step-major; the slot layout is documented in csrc/attention.cu);
+ * this copies the table of the last such launch to `host` (synchronous).
+ * slots and steps must equal the two constants. */
+#define H3DIT_ATTN_STAMP_SLOTS 32
+#define H3DIT_ATTN_STAMP_STEPS 300
+h3dit_status h3dit_attention_stamps(uint64_t *host, int32_t slots, int32_t steps);
+
 #ifdef __cplusplus
 }
 #endif
