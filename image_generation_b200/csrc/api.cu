@@ -383,6 +383,7 @@ h3dit_status run_linear(h3dit_ctx *ctx, int epi, const void *a, const void *w, i
   if (m < 0 || n <= 0 || k <= 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "bad shape %d x %d x %d", m, n, k);
   if (k % kGemmBK || n % 32)
     return ctx->fail(H3DIT_ERR_UNSUPPORTED, "linear needs k %% 64 == 0 and n %% 32 == 0 (k=%d n=%d)", k, n);
+  if (m == 0) return H3DIT_OK;  // no rows: no work, and the data pointers are not examined
   if (!a || !w || (!scatter && (!out || !aligned16(out))) || !aligned16(a) || !aligned16(w))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "linear: NULL or misaligned pointer");
   if (epi == H3DIT_EPI_GATED_RESIDUAL && (!gate || !aligned16(gate)))
@@ -418,7 +419,6 @@ h3dit_status run_linear(h3dit_ctx *ctx, int epi, const void *a, const void *w, i
       for (int g = 0; g < scatter->ranks; ++g) p.scatter[g] = scatter->ptr[g];
     }
   }
-  if (m == 0) return H3DIT_OK;
   // More than one 128-row block: 256 x 256 tiles on CTA pairs, which halves
   // the W traffic per SM; a single row block stays on the one-CTA kernel.
   const int max_pairs = H3_GEMM_PAIR && m > kGemmBM ? gemm_pair_max_clusters(epi) : 0;
@@ -483,6 +483,7 @@ h3dit_status run_linear_mx(h3dit_ctx *ctx, int epi, const void *a, const void *a
   if (m < 0 || n <= 0 || k <= 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "bad shape %d x %d x %d", m, n, k);
   if (k % kGemmMxBK || n % kGemmMxBN)
     return ctx->fail(H3DIT_ERR_UNSUPPORTED, "MXFP8 linear needs k and n multiples of 128 (k=%d n=%d)", k, n);
+  if (m == 0) return H3DIT_OK;  // no rows: no work, and the data pointers are not examined
   if (!a || !a_sf || !w || !w_sf || !out || !aligned16(a) || !aligned16(a_sf) || !aligned16(w) ||
       !aligned16(w_sf) || !aligned16(out))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "MXFP8 linear: NULL or misaligned pointer");
@@ -512,7 +513,6 @@ h3dit_status run_linear_mx(h3dit_ctx *ctx, int epi, const void *a, const void *a
     p.sec[1] = sec[1];
     p.sec[2] = sec[2];
   }
-  if (m == 0) return H3DIT_OK;
   const bool wide = w_sf_tiled && n % kGemmMxWideBN == 0;
   const int bn = wide ? kGemmMxWideBN : kGemmMxBN;
   CUtensorMap ta, tb;
@@ -555,13 +555,13 @@ h3dit_status run_attention(h3dit_ctx *ctx, const void *q, const void *k, const v
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "bad sequence batch");
   if (heads < 1 || heads > ctx->cfg.heads)
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "heads %d outside [1, %d]", heads, ctx->cfg.heads);
+  if (n == 0) return H3DIT_OK;  // no tokens: no work, and the data pointers are not examined
   if (!q || !k || !v || (!scatter && (!o || !aligned16(o))) || !aligned16(q) || !aligned16(k) ||
       !aligned16(v))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "attention: NULL or misaligned pointer");
   const int I = heads * ctx->cfg.head_dim;
   if (ld < I || ld % 8 || ldo < I || ldo % 8)
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "attention: row strides must be >= heads*head_dim and multiples of 8");
-  if (n == 0) return H3DIT_OK;
   CUtensorMap tq, tk, tv;
   h3dit_status st;
   const int rows = n * batch;
@@ -1070,17 +1070,16 @@ h3dit_status h3dit_rmsnorm_modulate(h3dit_ctx *ctx, const float *x, const float 
                                     void *cuda_stream) {
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
   if (n < 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "n < 0");
+  if (n == 0) return H3DIT_OK;
   if (!x || !shift || !scale || !xm_out || !aligned16(x) || !aligned16(shift) ||
       !aligned16(scale) || !aligned16(xm_out))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "NULL or misaligned pointer");
-  if (n == 0) return H3DIT_OK;
   return run_rmsnorm(ctx, x, shift, scale, xm_out, n, static_cast<cudaStream_t>(cuda_stream));
 }
 
 h3dit_status h3dit_rope_table(h3dit_ctx *ctx, const h3dit_grid *grids, int32_t n_grids,
                               int32_t n_txt, float *table_out, void *cuda_stream) {
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
-  if (!table_out) return ctx->fail(H3DIT_ERR_INVALID_ARG, "table_out is NULL");
   if (n_txt < 0 || n_grids < 0 || n_grids > kMaxGrids || (n_grids > 0 && !grids))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "bad grids");
   long long n = n_txt;
@@ -1090,6 +1089,7 @@ h3dit_status h3dit_rope_table(h3dit_ctx *ctx, const h3dit_grid *grids, int32_t n
     n += static_cast<long long>(grids[g].height) * grids[g].width;
   }
   if (n == 0) return H3DIT_OK;
+  if (!table_out) return ctx->fail(H3DIT_ERR_INVALID_ARG, "table_out is NULL");
   if (n > (1LL << 30)) return ctx->fail(H3DIT_ERR_INVALID_ARG, "too many tokens");
   return rope_table_into(ctx, grids, n_grids, n_txt, static_cast<int>(n), table_out,
                          static_cast<cudaStream_t>(cuda_stream));
@@ -1181,14 +1181,15 @@ h3dit_status h3dit_attention_heads(h3dit_ctx *ctx, int32_t heads, const void *q,
 }
 
 namespace {
+// Counts first; with no tokens the data pointers are not examined.
 h3dit_status check_sp(h3dit_ctx *ctx, const void *a, const void *b, int n_local, int ranks) {
-  if (!a || !b || !aligned16(a) || !aligned16(b))
-    return ctx->fail(H3DIT_ERR_INVALID_ARG, "sequence parallel re-layout: NULL or misaligned pointer");
   if (n_local < 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "n_local < 0");
   if (ranks < 1 || ctx->cfg.heads % ranks)
     return ctx->fail(H3DIT_ERR_UNSUPPORTED, "%d ranks do not divide %d heads", ranks, ctx->cfg.heads);
   if ((ctx->inner() / ranks) % 8)
     return ctx->fail(H3DIT_ERR_UNSUPPORTED, "a head group's width is not a multiple of 8");
+  if (n_local > 0 && (!a || !b || !aligned16(a) || !aligned16(b)))
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "sequence parallel re-layout: NULL or misaligned pointer");
   return H3DIT_OK;
 }
 }  // namespace
@@ -1218,12 +1219,14 @@ h3dit_status h3dit_sp_unpack_o(h3dit_ctx *ctx, const void *recv, int32_t n_local
 }
 
 namespace {
-h3dit_status check_scatter(h3dit_ctx *ctx, void *const *dst, int ranks, int rank) {
+h3dit_status check_scatter(h3dit_ctx *ctx, void *const *dst, int ranks, int rank, int count) {
   if (ranks < 1 || ranks > kMaxScatterRanks)
     return ctx->fail(H3DIT_ERR_UNSUPPORTED, "%d ranks: the fused exchange addresses 1 .. %d",
                      ranks, kMaxScatterRanks);
   if (rank < 0 || rank >= ranks)
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "rank %d outside [0, %d)", rank, ranks);
+  if (count < 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "negative token count");
+  if (count == 0) return H3DIT_OK;  // no tokens: the destinations are not examined
   if (!dst) return ctx->fail(H3DIT_ERR_INVALID_ARG, "NULL destination array");
   for (int g = 0; g < ranks; ++g)
     if (!dst[g] || !aligned16(dst[g]))
@@ -1237,9 +1240,9 @@ h3dit_status h3dit_sp_qkv_scatter(h3dit_ctx *ctx, const void *xm, int32_t n_loca
                                   int32_t ranks, int32_t rank, void *cuda_stream) {
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
   if (ctx->vae) return ctx->fail(H3DIT_ERR_UNSUPPORTED, "a decoder context runs h3dit_vae_decode");
-  h3dit_status st = check_scatter(ctx, recv, ranks, rank);
+  h3dit_status st = check_scatter(ctx, recv, ranks, rank, n_local);
   if (st) return st;
-  if ((st = check_sp(ctx, xm, w_qkv, n_local, ranks))) return st;
+  if ((st = check_sp(ctx, xm, w_qkv, n_local, ranks)) || n_local == 0) return st;
   const ScatterTargets sc{recv, ranks, rank};
   const int I = ctx->inner();
   return run_linear(ctx, H3DIT_EPI_QKV_ROPE, xm, w_qkv, n_local, 3 * I, ctx->cfg.hidden, nullptr,
@@ -1252,9 +1255,9 @@ h3dit_status h3dit_sp_attention_scatter(h3dit_ctx *ctx, const void *qkv, int32_t
                                         void *cuda_stream) {
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
   if (ctx->vae) return ctx->fail(H3DIT_ERR_UNSUPPORTED, "a decoder context runs h3dit_vae_decode");
-  h3dit_status st = check_scatter(ctx, o, ranks, rank);
+  h3dit_status st = check_scatter(ctx, o, ranks, rank, n_total);
   if (st) return st;
-  if ((st = check_sp(ctx, qkv, o[0], n_total, ranks))) return st;
+  if ((st = check_sp(ctx, qkv, n_total ? o[0] : nullptr, n_total, ranks)) || n_total == 0) return st;
   if (n_total % ranks)
     return ctx->fail(H3DIT_ERR_UNSUPPORTED, "%d tokens do not split over %d ranks", n_total, ranks);
   const ScatterTargets sc{o, ranks, rank};
@@ -1530,10 +1533,10 @@ h3dit_status h3dit_layernorm(h3dit_ctx *ctx, const float *x, const float *gain, 
                              void *out, int32_t n, void *cuda_stream) {
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
   if (n < 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "n < 0");
+  if (n == 0) return H3DIT_OK;
   if (!x || !gain || !bias || !out || !aligned16(x) || !aligned16(gain) || !aligned16(bias) ||
       !aligned16(out))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "NULL or misaligned pointer");
-  if (n == 0) return H3DIT_OK;
   return run_layernorm(ctx, x, gain, bias, out, n, static_cast<cudaStream_t>(cuda_stream));
 }
 
@@ -1564,6 +1567,7 @@ h3dit_status h3dit_mx_quantize(h3dit_ctx *ctx, const void *src, int32_t rows, in
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
   if (rows < 0 || k <= 0 || k % 128)
     return ctx->fail(H3DIT_ERR_UNSUPPORTED, "MXFP8 quantization needs k a multiple of 128");
+  if (rows == 0) return H3DIT_OK;
   if (!src || !dst || !sf || !aligned16(src) || !aligned16(dst))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "NULL or misaligned pointer");
   Launch L(ctx, H3DIT_KERNEL_MX_QUANTIZE, static_cast<cudaStream_t>(cuda_stream));
@@ -1623,10 +1627,10 @@ h3dit_status h3dit_rmsnorm_modulate_mx(h3dit_ctx *ctx, const float *x, const flo
   if (!ctx) return H3DIT_ERR_INVALID_ARG;
   if (n < 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "n < 0");
   if (ctx->cfg.hidden % 128) return ctx->fail(H3DIT_ERR_UNSUPPORTED, "MXFP8 needs hidden % 128 == 0");
+  if (n == 0) return H3DIT_OK;
   if (!x || !shift || !scale || !out || !out_sf || !aligned16(x) || !aligned16(shift) ||
       !aligned16(scale) || !aligned16(out))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "NULL or misaligned pointer");
-  if (n == 0) return H3DIT_OK;
   return run_rmsnorm(ctx, x, shift, scale, out, n, static_cast<cudaStream_t>(cuda_stream),
                      static_cast<uint8_t *>(out_sf));
 }

@@ -45,6 +45,12 @@ typedef int32_t h3dit_status;
 #define H3DIT_ERR_CUDA (-4)        /* a CUDA runtime or launch error */
 #define H3DIT_ERR_TIMEOUT (-5)     /* a kernel's bounded wait gave up (see h3dit_sync_status) */
 
+/* Empty inputs: a stage call whose row or token count is 0 (m of the
+ * linears, n of the norms and the attention, n_local / n_total of the
+ * sequence-parallel calls, rows of h3dit_mx_quantize, an empty RoPE table)
+ * checks its counts and shape arguments, then returns H3DIT_OK without
+ * launching anything or examining its data pointers, which may be NULL. */
+
 /* Epilogues of h3dit_linear (steps a4, a6/a9, a8 of the block). */
 #define H3DIT_EPI_STORE 0          /* out bf16 [m, n] = a w^T                          */
 #define H3DIT_EPI_QKV_ROPE 1       /* as STORE, RoPE on columns < 2*heads*head_dim    */
