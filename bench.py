@@ -616,11 +616,24 @@ def block_timings(dh: int) -> dict:
     return out
 
 
-def streaming_timings(tw, blocks, x_txt, x_img, grids, dh, residents=(24, 8), steps=2,
+def streamed_set(k: int, placement: str) -> set:
+    """Which of the L blocks stream from the host when k stay resident:
+    "tail" streams blocks k .. L-1; "spread" spaces the L - k streamed blocks
+    evenly through the step, so that each one's copy overlaps the compute of
+    the resident blocks around it as well as of the previous streamed block."""
+    if placement == "tail":
+        return set(range(k, L))
+    m = L - k
+    return {l for l in range(L) if (l + 1) * m // L - l * m // L == 1}
+
+
+def streaming_timings(tw, blocks, x_txt, x_img, grids, dh,
+                      residents=((24, "tail"), (24, "spread"), (8, "spread")), steps=2,
                       host_copies=4):
-    """The 50-block 4096^2 step with only the first k blocks' weights on the
-    device and the rest streamed from pinned host memory through two staging
-    slots (h3dit_attach_staging). The host blocks cycle through
+    """The 50-block 4096^2 step with only k blocks' weights on the device
+    (placed as streamed_set says) and the rest streamed from pinned host
+    memory through two staging slots (h3dit_attach_staging). The host blocks
+    cycle through
     `host_copies` distinct pinned copies of the model's own blocks (the bytes
     moved per step are the same as with 50 - k distinct blocks; the step's
     output is not compared here - the tests check streamed steps bit for bit
@@ -634,8 +647,10 @@ def streaming_timings(tw, blocks, x_txt, x_img, grids, dh, residents=(24, 8), st
             for i in range(host_copies)]
     block_bytes = sum(v.numel() * v.element_size() for v in host[0].values())
     out = {}
-    for k in residents:
-        mixed = [blocks[l] if l < k else host[l % host_copies] for l in range(L)]
+    for k, placement in residents:
+        streamed = streamed_set(k, placement)
+        assert len(streamed) == L - k
+        mixed = [host[l % host_copies] if l in streamed else blocks[l] for l in range(L)]
         ctx = Hb.Context(Hb.make_config(D, H, dh, F, L, N_TOK), tw, mixed)
         ctx.attach_staging()
         ts = timesteps(steps + 1)
@@ -651,7 +666,8 @@ def streaming_timings(tw, blocks, x_txt, x_img, grids, dh, residents=(24, 8), st
             raise RuntimeError(f"streamed step failed (k={k})")
         ms = e0.elapsed_time(e1) / steps
         moved = (L - k) * block_bytes
-        out[f"resident_{k}"] = {"ms_per_step": round(ms, 1), "streamed_blocks": L - k,
+        name = f"resident_{k}" if placement == "tail" else f"resident_{k}_{placement}"
+        out[name] = {"ms_per_step": round(ms, 1), "streamed_blocks": L - k, "placement": placement,
                                 "h2d_bytes_per_step": moved,
                                 "h2d_gbs": round(moved / ms / 1e6, 1)}
         ctx.close()

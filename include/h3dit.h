@@ -153,7 +153,11 @@ void h3dit_destroy(h3dit_ctx *ctx);
  * host block's AdaLN projection is computed from its slot just before it
  * runs. Results are bit-identical to the same weights held on the device.
  * Every call is still ordered on its `cuda_stream`: the copy stream forks
- * from it at entry and joins it at exit (so a step can be graph-captured). */
+ * from it at entry and joins it at exit (so a step can be graph-captured).
+ * Placement: a block's copy can overlap only the compute that runs between
+ * its slot's release and its own turn. With host blocks spaced evenly
+ * through the step (resident blocks between them), each copy overlaps two or
+ * more blocks of compute; with the host blocks in one run, only one. */
 
 /* Bytes of staging memory h3dit_attach_staging needs for `cfg` (two slots of
  * one block's weights and a small pointer table), or 0 if `cfg` is invalid. */
