@@ -368,10 +368,12 @@ h3dit_status encode_heads(h3dit_ctx *ctx, CUtensorMap *m, const void *base, int 
   return H3DIT_OK;
 }
 
-// Destination buffers of a fused Ulysses exchange, one per rank.
+// Destination buffers of a fused Ulysses exchange, one per rank (and, for
+// an MXFP8 attention output, each rank's scale array).
 struct ScatterTargets {
   void *const *ptr;
   int ranks, rank;
+  void *const *sf = nullptr;
 };
 
 h3dit_status run_linear(h3dit_ctx *ctx, int epi, const void *a, const void *w, int m, int n,
@@ -477,15 +479,16 @@ h3dit_status encode_fp8(h3dit_ctx *ctx, CUtensorMap *m, const void *base, uint64
 h3dit_status run_linear_mx(h3dit_ctx *ctx, int epi, const void *a, const void *a_sf, const void *w,
                            const void *w_sf, int m, int n, int k, void *out, long long ldo,
                            void *out_sf, const float *gate, const float *rope, cudaStream_t s,
-                           const void *w_sf_tiled = nullptr) {
+                           const void *w_sf_tiled = nullptr,
+                           const ScatterTargets *scatter = nullptr) {
   if (epi < H3DIT_EPI_STORE || epi > H3DIT_EPI_GATED_RESIDUAL)
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "unknown epilogue %d", epi);
   if (m < 0 || n <= 0 || k <= 0) return ctx->fail(H3DIT_ERR_INVALID_ARG, "bad shape %d x %d x %d", m, n, k);
   if (k % kGemmMxBK || n % kGemmMxBN)
     return ctx->fail(H3DIT_ERR_UNSUPPORTED, "MXFP8 linear needs k and n multiples of 128 (k=%d n=%d)", k, n);
   if (m == 0) return H3DIT_OK;  // no rows: no work, and the data pointers are not examined
-  if (!a || !a_sf || !w || !w_sf || !out || !aligned16(a) || !aligned16(a_sf) || !aligned16(w) ||
-      !aligned16(w_sf) || !aligned16(out))
+  if (!a || !a_sf || !w || !w_sf || (!scatter && (!out || !aligned16(out))) || !aligned16(a) ||
+      !aligned16(a_sf) || !aligned16(w) || !aligned16(w_sf))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "MXFP8 linear: NULL or misaligned pointer");
   if (epi == H3DIT_EPI_GATED_RESIDUAL && (!gate || !aligned16(gate)))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "gated residual needs a 16-byte aligned gate");
@@ -512,6 +515,13 @@ h3dit_status run_linear_mx(h3dit_ctx *ctx, int epi, const void *a, const void *a
     p.sec[0] = sec[0];
     p.sec[1] = sec[1];
     p.sec[2] = sec[2];
+    if (scatter) {  // as in run_linear: the first Ulysses all-to-all in the epilogue
+      p.scatter_ranks = scatter->ranks;
+      p.scatter_rank = scatter->rank;
+      p.scatter_inner = I;
+      p.scatter_cols = I / scatter->ranks;
+      for (int g = 0; g < scatter->ranks; ++g) p.scatter[g] = scatter->ptr[g];
+    }
   }
   const bool wide = w_sf_tiled && n % kGemmMxWideBN == 0;
   const int bn = wide ? kGemmMxWideBN : kGemmMxBN;
@@ -579,6 +589,18 @@ h3dit_status run_attention(h3dit_ctx *ctx, const void *q, const void *k, const v
   p.o_sf = static_cast<uint8_t *>(o_sf);
   if (o_sf && (ldo != I || I % 128 || !aligned16(o_sf)))
     return ctx->fail(H3DIT_ERR_INVALID_ARG, "MXFP8 attention output needs ld_o == heads*head_dim, a multiple of 128");
+  const bool out_mx = o_sf != nullptr || (scatter && scatter->sf);
+  if (scatter && scatter->sf) {
+    // an MXFP8 output scattered to [n / ranks, ld_o] E4M3 rows of every head
+    if (ldo != ctx->inner() || ldo % 128)
+      return ctx->fail(H3DIT_ERR_INVALID_ARG,
+                       "MXFP8 scattered output needs ld_o == heads*head_dim, a multiple of 128");
+    for (int g = 0; g < scatter->ranks; ++g) {
+      if (!scatter->sf[g] || !aligned16(scatter->sf[g]))
+        return ctx->fail(H3DIT_ERR_INVALID_ARG, "scale array of rank %d is NULL or misaligned", g);
+      p.o_sf_scatter[g] = static_cast<uint8_t *>(scatter->sf[g]);
+    }
+  }
   if (scatter) {
     // rank r's rows of the sequence go to its [n / ranks, ld_o] output, at
     // this rank's head group's columns
@@ -588,7 +610,7 @@ h3dit_status run_attention(h3dit_ctx *ctx, const void *q, const void *k, const v
     for (int g = 0; g < scatter->ranks; ++g) p.o_scatter[g] = scatter->ptr[g];
   }
   Launch L(ctx, H3DIT_KERNEL_ATTENTION, s);
-  return ctx->cuda(launch_attention(tq, tk, tv, p, ctx->cfg.head_dim, heads, o_sf != nullptr, s),
+  return ctx->cuda(launch_attention(tq, tk, tv, p, ctx->cfg.head_dim, heads, out_mx, s),
                    "attention launch");
 }
 
@@ -1261,6 +1283,46 @@ h3dit_status h3dit_sp_attention_scatter(h3dit_ctx *ctx, const void *qkv, int32_t
   if (n_total % ranks)
     return ctx->fail(H3DIT_ERR_UNSUPPORTED, "%d tokens do not split over %d ranks", n_total, ranks);
   const ScatterTargets sc{o, ranks, rank};
+  const int I = ctx->inner(), cw = I / ranks;
+  const uint16_t *q = static_cast<const uint16_t *>(qkv);
+  return run_attention(ctx, q, q + cw, q + 2 * cw, 3 * cw, nullptr, I, n_total,
+                       static_cast<cudaStream_t>(cuda_stream), nullptr, ctx->cfg.heads / ranks, 1,
+                       &sc);
+}
+
+h3dit_status h3dit_sp_qkv_scatter_mx(h3dit_ctx *ctx, const void *xq, const void *xq_sf,
+                                     int32_t n_local, int32_t block, const float *rope_rows,
+                                     void *const *recv, int32_t ranks, int32_t rank,
+                                     void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (!ctx->mx()) return ctx->fail(H3DIT_ERR_UNSUPPORTED, "the context is not MXFP8");
+  if (block < 0 || block >= ctx->cfg.n_blocks)
+    return ctx->fail(H3DIT_ERR_INVALID_ARG, "block %d outside [0, %d)", block, ctx->cfg.n_blocks);
+  h3dit_status st = check_scatter(ctx, recv, ranks, rank, n_local);
+  if (st) return st;
+  if ((st = check_sp(ctx, xq, xq_sf, n_local, ranks)) || n_local == 0) return st;
+  const MxWeights &o = ctx->L.wq_off;
+  const int I = ctx->inner();
+  const ScatterTargets sc{recv, ranks, rank};
+  return run_linear_mx(ctx, H3DIT_EPI_QKV_ROPE, xq, xq_sf, ctx->wq(block, o.qkv),
+                       ctx->wq(block, o.qkv_sf), n_local, 3 * I, ctx->cfg.hidden, nullptr, 3 * I,
+                       nullptr, nullptr, rope_rows, static_cast<cudaStream_t>(cuda_stream),
+                       o.qkv_sft == kNoTiled ? nullptr : ctx->wq(block, o.qkv_sft), &sc);
+}
+
+h3dit_status h3dit_sp_attention_scatter_mx(h3dit_ctx *ctx, const void *qkv, int32_t n_total,
+                                           void *const *o, void *const *o_sf, int32_t ranks,
+                                           int32_t rank, void *cuda_stream) {
+  if (!ctx) return H3DIT_ERR_INVALID_ARG;
+  if (ctx->vae) return ctx->fail(H3DIT_ERR_UNSUPPORTED, "a decoder context runs h3dit_vae_decode");
+  h3dit_status st = check_scatter(ctx, o, ranks, rank, n_total);
+  if (st) return st;
+  if (n_total > 0 && !o_sf) return ctx->fail(H3DIT_ERR_INVALID_ARG, "NULL scale array list");
+  if ((st = check_sp(ctx, qkv, n_total ? o[0] : nullptr, n_total, ranks)) || n_total == 0)
+    return st;
+  if (n_total % ranks)
+    return ctx->fail(H3DIT_ERR_UNSUPPORTED, "%d tokens do not split over %d ranks", n_total, ranks);
+  const ScatterTargets sc{o, ranks, rank, o_sf};
   const int I = ctx->inner(), cw = I / ranks;
   const uint16_t *q = static_cast<const uint16_t *>(qkv);
   return run_attention(ctx, q, q + cw, q + 2 * cw, 3 * cw, nullptr, I, n_total,

@@ -420,16 +420,22 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float inv_l = 1.f / l;
       const int qrow = q0 + t * BQ + row;  // within the sequence
       const size_t grow = static_cast<size_t>(seq0) + qrow;
-      uint16_t *dst;
-      if (p.o_scatter_ranks == 0) {
-        dst = static_cast<uint16_t *>(p.o) + grow * p.ldo + head * DH;
-      } else {
-        // the second Ulysses all-to-all: this row belongs to rank grow / rows
-        const int owner = static_cast<int>(grow / static_cast<size_t>(p.o_rows_per_rank));
-        const size_t local = grow - static_cast<size_t>(owner) * p.o_rows_per_rank;
-        dst = static_cast<uint16_t *>(p.o_scatter[owner < kMaxScatterRanks ? owner : 0]) +
-              local * p.ldo + p.o_col0 + head * DH;
+      // where this row's output goes: row grow of o, or, with the second
+      // Ulysses all-to-all fused in, row grow % rows of the output of the
+      // rank that holds the token, at this rank's head-group columns
+      void *obase = p.o;
+      uint8_t *sfbase = p.o_sf;
+      size_t orow = grow;
+      int col0 = head * DH;
+      if (p.o_scatter_ranks != 0) {
+        int owner = static_cast<int>(grow / static_cast<size_t>(p.o_rows_per_rank));
+        owner = owner < kMaxScatterRanks ? owner : 0;  // only rows past n reach beyond
+        orow = grow - static_cast<size_t>(owner) * p.o_rows_per_rank;
+        col0 += p.o_col0;
+        obase = p.o_scatter[owner];
+        sfbase = p.o_sf_scatter[owner];
       }
+      uint16_t *dst = static_cast<uint16_t *>(obase) + orow * p.ldo + col0;
 #pragma unroll
       for (int c = 0; c < DH / 32; ++c) {
         uint32_t r[32];
@@ -441,13 +447,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * inv_l;
             uint32_t q[8];
             const uint32_t sb = mx_quant32(v, q);
-            uint8_t *d8 = static_cast<uint8_t *>(p.o) + grow * p.ldo +
-                          head * DH + 32 * c;
+            uint8_t *d8 = static_cast<uint8_t *>(obase) + orow * p.ldo + col0 + 32 * c;
             st_global_v4(d8, q[0], q[1], q[2], q[3]);
             st_global_v4(d8 + 16, q[4], q[5], q[6], q[7]);
-            p.o_sf[mx_sf_offset(static_cast<int>(grow), (head * DH) / 32 + c,
-                                static_cast<int>(p.ldo / 128))] =
-                static_cast<uint8_t>(sb);
+            sfbase[mx_sf_offset(static_cast<int>(orow), col0 / 32 + c,
+                                static_cast<int>(p.ldo / 128))] = static_cast<uint8_t>(sb);
           }
           continue;
         }

@@ -120,8 +120,10 @@ struct AttnParams {
   uint8_t *o_sf;          // MXFP8 output: scales of o [n, heads*head_dim]
   // The second Ulysses all-to-all fused in (o_scatter_ranks > 0): output row
   // t goes to o_scatter[t / o_rows_per_rank] at row t % o_rows_per_rank,
-  // column o_col0 + head * head_dim, with row stride ldo; `o` is unused.
+  // column o_col0 + head * head_dim, with row stride ldo (and its MXFP8
+  // scales to o_sf_scatter of the same rank); `o` and `o_sf` are unused.
   void *o_scatter[kMaxScatterRanks];
+  uint8_t *o_sf_scatter[kMaxScatterRanks];  // MXFP8 output: the owners' scale arrays
   int o_scatter_ranks;
   int o_rows_per_rank;
   int o_col0;

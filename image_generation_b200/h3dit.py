@@ -138,6 +138,9 @@ def _load() -> C.CDLL:
         "h3dit_sp_unpack_o": (i32, [p, p, i32, i32, p, p]),
         "h3dit_sp_qkv_scatter": (i32, [p, p, i32, p, p, C.POINTER(p), i32, i32, p]),
         "h3dit_sp_attention_scatter": (i32, [p, p, i32, C.POINTER(p), i32, i32, p]),
+        "h3dit_sp_qkv_scatter_mx": (i32, [p, p, p, i32, i32, p, C.POINTER(p), i32, i32, p]),
+        "h3dit_sp_attention_scatter_mx": (i32, [p, p, i32, C.POINTER(p), C.POINTER(p), i32, i32,
+                                                p]),
         "h3dit_ipc_get_handle": (i32, [p, p, C.POINTER(C.c_uint64)]),
         "h3dit_ipc_open": (i32, [p, C.c_uint64, C.POINTER(p)]),
         "h3dit_ipc_close": (i32, [p, C.c_uint64]),
@@ -379,11 +382,17 @@ class Context:
 
     def empty(self, shape, kind: str):
         """A device buffer for the sequence-parallel driver: "act" and
-        "exchange" (activations other ranks write into) are bf16, "f32" and
-        "rope" are fp32."""
+        "exchange" (activations other ranks write into) are bf16; "fp8",
+        "exchange_fp8" (E4M3 codes) and "sf", "exchange_sf" (MXFP8 scale
+        bytes) are uint8; "f32" and "rope" are fp32."""
         import torch
 
-        dt = torch.bfloat16 if kind in ("act", "exchange") else torch.float32
+        if kind in ("act", "exchange"):
+            dt = torch.bfloat16
+        elif kind in ("fp8", "exchange_fp8", "sf", "exchange_sf"):
+            dt = torch.uint8
+        else:
+            dt = torch.float32
         return torch.empty(*shape, dtype=dt, device="cuda")
 
     def attention_heads(self, heads: int, q, k, v, ld_qkv: int, o, ld_o: int, n: int,
@@ -423,6 +432,31 @@ class Context:
         self._check(lib.h3dit_sp_attention_scatter(self.handle, _ptr(qkv_recv),
                                                    qkv_recv.shape[0], arr, len(o_ptrs), rank,
                                                    _stream(stream)))
+
+    def sp_qkv_scatter_mx(self, xq, xq_sf, block: int, rope_rows, recv_ptrs: Sequence[int],
+                          rank: int, stream=None) -> None:
+        """sp_qkv_scatter for an MXFP8 context: this rank's quantized rows
+        xq [n_local, D] (E4M3) with scales xq_sf, times the context's
+        quantized QKV weights of `block`."""
+        arr = (C.c_void_p * len(recv_ptrs))(*recv_ptrs)
+        self._check(lib.h3dit_sp_qkv_scatter_mx(self.handle, _ptr(xq), _ptr(xq_sf), xq.shape[0],
+                                                block, _ptr(rope_rows), arr, len(recv_ptrs), rank,
+                                                _stream(stream)))
+
+    def sp_attention_scatter_mx(self, qkv_recv, o_ptrs: Sequence[int], o_sf_ptrs: Sequence[int],
+                                rank: int, stream=None) -> None:
+        """sp_attention_scatter with MXFP8 output rows: E4M3 into o_ptrs[r]
+        ([N / ranks, I]) and scales into o_sf_ptrs[r]."""
+        if len(o_sf_ptrs) != len(o_ptrs):
+            raise H3DitError(H3DIT_ERR_INVALID_ARG, "one scale array per output")
+        arr = (C.c_void_p * len(o_ptrs))(*o_ptrs)
+        sfa = (C.c_void_p * len(o_sf_ptrs))(*o_sf_ptrs)
+        self._check(lib.h3dit_sp_attention_scatter_mx(self.handle, _ptr(qkv_recv),
+                                                      qkv_recv.shape[0], arr, sfa, len(o_ptrs),
+                                                      rank, _stream(stream)))
+
+    def mx_scale_bytes(self, rows: int, k: int) -> int:
+        return mx_scale_bytes(rows, k)
 
     def block_forward(self, block: int, t: float, x_img, grids, x_txt, mod=None,
                       stream=None) -> None:

@@ -42,6 +42,7 @@ from typing import Callable, Sequence
 H3DIT_EPI_QKV_ROPE = 1
 H3DIT_EPI_GELU = 2
 H3DIT_EPI_GATED_RESIDUAL = 3
+H3DIT_LINEAR_OUT, H3DIT_LINEAR_FFN1, H3DIT_LINEAR_FFN2 = 1, 2, 3
 
 
 class UlyssesRank:
@@ -117,10 +118,16 @@ class FusedUlyssesRank:
     the Q|K|V of this rank's heads from every rank's QKV GEMM, and `o`
     [N/P, I] receives this rank's token rows of the attention output from
     every rank's attention. `connect` takes every rank's `recv` and `o`
-    device addresses in rank order (its own included)."""
+    device addresses in rank order (its own included).
+
+    With mx=True the block runs the MXFP8 linears of an MXFP8 context (the
+    context's quantized weights, so the stages take the block's index): the
+    rows are quantized by the MXFP8 RMSNorm, `o` holds E4M3 codes and
+    `o_sf` their scales, which every rank's attention writes too; `recv`
+    stays bf16."""
 
     def __init__(self, ops, rank: int, world: int, n_total: int, hidden: int, heads: int,
-                 head_dim: int, ffn: int, max_ranks: int = 8):
+                 head_dim: int, ffn: int, max_ranks: int = 8, mx: bool = False):
         if not 1 <= world <= max_ranks:
             raise ValueError(f"the fused exchange addresses 1 .. {max_ranks} ranks, not {world}")
         if n_total % world:
@@ -132,52 +139,89 @@ class FusedUlyssesRank:
         self.D, self.H, self.dh, self.F = hidden, heads, head_dim, ffn
         self.I = heads * head_dim
         self.cw = self.I // world
+        self.mx = mx
         e = ops.empty
-        self.xm = e((self.n, hidden), "act")
         self.recv = e((n_total, 3 * self.cw), "exchange")  # written by every rank
-        self.o = e((self.n, self.I), "exchange")            # written by every rank
-        self.u = e((self.n, ffn), "act")
+        if mx:
+            sf = ops.mx_scale_bytes
+            self.xm = e((self.n, hidden), "fp8")
+            self.xm_sf = e((sf(self.n, hidden),), "sf")
+            self.o = e((self.n, self.I), "exchange_fp8")          # written by every rank
+            self.o_sf = e((sf(self.n, self.I),), "exchange_sf")   # written by every rank
+            self.u = e((self.n, ffn), "fp8")
+            self.u_sf = e((sf(self.n, ffn),), "sf")
+        else:
+            self.xm = e((self.n, hidden), "act")
+            self.o = e((self.n, self.I), "exchange")            # written by every rank
+            self.u = e((self.n, ffn), "act")
         self.recv_ptrs: list | None = None
         self.o_ptrs: list | None = None
+        self.o_sf_ptrs: list | None = None
+
+    def exchanged(self) -> list:
+        """The buffers other ranks write into, in the order connect takes
+        their addresses."""
+        return [self.recv, self.o] + ([self.o_sf] if self.mx else [])
 
     def rows(self):
         return slice(self.rank * self.n, (self.rank + 1) * self.n)
 
-    def connect(self, recv_ptrs: Sequence[int], o_ptrs: Sequence[int]) -> None:
+    def connect(self, recv_ptrs: Sequence[int], o_ptrs: Sequence[int],
+                o_sf_ptrs: Sequence[int] | None = None) -> None:
         if len(recv_ptrs) != self.world or len(o_ptrs) != self.world:
             raise ValueError("one receive and one output address per rank")
+        if self.mx and (o_sf_ptrs is None or len(o_sf_ptrs) != self.world):
+            raise ValueError("one scale-array address per rank")
         self.recv_ptrs, self.o_ptrs = list(recv_ptrs), list(o_ptrs)
+        self.o_sf_ptrs = None if o_sf_ptrs is None else list(o_sf_ptrs)
 
-    def qkv_scatter(self, x, mod, w, rope_rows) -> None:
+    def qkv_scatter(self, x, mod, w, rope_rows, block: int = 0) -> None:
         """RMSNorm + modulate, then QKV + RoPE with the first exchange fused
         in: every rank's `recv` gets this rank's rows of its head group."""
+        if self.mx:
+            self.ops.rmsnorm_modulate_mx(x, mod[0], mod[1], self.xm, self.xm_sf)
+            self.ops.sp_qkv_scatter_mx(self.xm, self.xm_sf, block, rope_rows, self.recv_ptrs,
+                                       self.rank)
+            return
         self.ops.rmsnorm_modulate(x, mod[0], mod[1], self.xm)
         self.ops.sp_qkv_scatter(self.xm, w["w_qkv"], rope_rows, self.recv_ptrs, self.rank)
 
     def attention_scatter(self) -> None:
         """Attention of this rank's heads over all tokens, with the second
         exchange fused in: every rank's `o` gets its rows for these heads."""
+        if self.mx:
+            self.ops.sp_attention_scatter_mx(self.recv, self.o_ptrs, self.o_sf_ptrs, self.rank)
+            return
         self.ops.sp_attention_scatter(self.recv, self.o_ptrs, self.rank)
 
-    def finish(self, x, mod, w) -> None:
+    def finish(self, x, mod, w, block: int = 0) -> None:
         ops = self.ops
+        if self.mx:
+            ops.block_linear_mx(block, H3DIT_LINEAR_OUT, self.o, self.o_sf, x, gate=mod[2])
+            ops.rmsnorm_modulate_mx(x, mod[3], mod[4], self.xm, self.xm_sf)
+            ops.block_linear_mx(block, H3DIT_LINEAR_FFN1, self.xm, self.xm_sf, self.u, self.u_sf)
+            ops.block_linear_mx(block, H3DIT_LINEAR_FFN2, self.u, self.u_sf, x, gate=mod[5])
+            return
         ops.linear(H3DIT_EPI_GATED_RESIDUAL, self.o, w["w_o"], x, gate=mod[2])
         ops.rmsnorm_modulate(x, mod[3], mod[4], self.xm)
         ops.linear(H3DIT_EPI_GELU, self.xm, w["w_ff1"], self.u)
         ops.linear(H3DIT_EPI_GATED_RESIDUAL, self.u, w["w_ff2"], x, gate=mod[5])
 
 
-def fused_block(rank: FusedUlyssesRank, x, mod, w, rope_rows, barrier: Callable) -> None:
-    """One block with the fused exchanges. barrier() must return only when
-    every rank's work so far has completed on its GPU: after the first stage
-    the attention reads what all ranks wrote, and after the second the
-    out-projection does; the next block's first stage then overwrites `recv`,
-    which every rank has finished reading by the second barrier."""
-    rank.qkv_scatter(x, mod, w, rope_rows)
+def fused_block(rank: FusedUlyssesRank, x, mod, w, rope_rows, barrier: Callable,
+                block: int = 0) -> None:
+    """One block with the fused exchanges (`block`: its index, which the
+    MXFP8 form uses to find the context's quantized weights). barrier() must
+    return only when every rank's work so far has completed on its GPU: after
+    the first stage the attention reads what all ranks wrote, and after the
+    second the out-projection does; the next block's first stage then
+    overwrites `recv`, which every rank has finished reading by the second
+    barrier."""
+    rank.qkv_scatter(x, mod, w, rope_rows, block)
     barrier()
     rank.attention_scatter()
     barrier()
-    rank.finish(x, mod, w)
+    rank.finish(x, mod, w, block)
 
 
 def connect_peers(rank: FusedUlyssesRank, ipc=None, group=None) -> list:
@@ -199,25 +243,22 @@ def connect_peers(rank: FusedUlyssesRank, ipc=None, group=None) -> list:
         h, off = ipc.handle(t)
         return h, off, t.data_ptr() - off  # the allocation's base in the owner
 
-    mine = (named(rank.recv), named(rank.o))
+    bufs = rank.exchanged()
+    mine = [named(t) for t in bufs]
     everyone = [None] * rank.world
     dist.all_gather_object(everyone, mine, group=group)
     bases: dict = {}
-    recv_ptrs, o_ptrs = [], []
-    for r, pair in enumerate(everyone):
-        if r == rank.rank:
-            recv_ptrs.append(rank.recv.data_ptr())
-            o_ptrs.append(rank.o.data_ptr())
-            continue
-        ptrs = []
-        for h, off, owner_base in pair:
+    cols: list = [[] for _ in bufs]  # per buffer, every rank's address
+    for r, names in enumerate(everyone):
+        for i, (h, off, owner_base) in enumerate(names):
+            if r == rank.rank:
+                cols[i].append(bufs[i].data_ptr())
+                continue
             key = (r, owner_base)  # one opening per allocation of each rank
             if key not in bases:
                 bases[key] = ipc.open(h)
-            ptrs.append(bases[key] + off)
-        recv_ptrs.append(ptrs[0])
-        o_ptrs.append(ptrs[1])
-    rank.connect(recv_ptrs, o_ptrs)
+            cols[i].append(bases[key] + off)
+    rank.connect(*cols)
     return list(bases.values())
 
 
@@ -265,12 +306,15 @@ class UlyssesStep:
     def __init__(self, ops, weights: Sequence[dict], rank: int, world: int, n_total: int,
                  hidden: int, heads: int, head_dim: int, ffn: int,
                  all_to_all: Callable | None = None, group=None, fused: bool = False,
-                 barrier: Callable | None = None, ipc=None):
+                 barrier: Callable | None = None, ipc=None, mx: bool = False):
         self.fused = fused
         self.peer_bases: list = []
+        if mx and not fused:
+            raise ValueError("the MXFP8 block runs with the fused exchanges")
         if fused:
             # collective: every rank constructs its step at the same point
-            self.r = FusedUlyssesRank(ops, rank, world, n_total, hidden, heads, head_dim, ffn)
+            self.r = FusedUlyssesRank(ops, rank, world, n_total, hidden, heads, head_dim, ffn,
+                                      mx=mx)
             self.peer_bases = connect_peers(self.r, ipc=ipc, group=group)
             self.barrier = barrier if barrier is not None else host_barrier(group)
         else:
@@ -294,7 +338,7 @@ class UlyssesStep:
         rope_rows = self.rope[self.r.rows()]
         for l, w in enumerate(self.weights):
             if self.fused:
-                fused_block(self.r, x, self.mod[l], w, rope_rows, self.barrier)
+                fused_block(self.r, x, self.mod[l], w, rope_rows, self.barrier, block=l)
             else:
                 block(self.r, x, self.mod[l], w, rope_rows, self.all_to_all)
 

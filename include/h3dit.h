@@ -316,6 +316,26 @@ h3dit_status h3dit_sp_attention_scatter(h3dit_ctx *ctx, const void *qkv, int32_t
                                         void *const *o, int32_t ranks, int32_t rank,
                                         void *cuda_stream);
 
+/* The same two fused exchanges for a context with H3DIT_PRECISION_MXFP8 (the
+ * MXFP8 block of h3dit_block_linear_mx, run over ranks).
+ * h3dit_sp_qkv_scatter_mx: as h3dit_sp_qkv_scatter, from this rank's
+ * quantized rows xq (device E4M3 [n_local, D]) and their scales xq_sf (the
+ * layout h3dit_rmsnorm_modulate_mx writes), with the context's quantized QKV
+ * weights of `block`; the receive buffers stay bf16.
+ * h3dit_sp_attention_scatter_mx: as h3dit_sp_attention_scatter, but each
+ * output row is written as MXFP8, the input h3dit_block_linear_mx's
+ * out-projection takes: E4M3 into o[t / n_local] (device [n_local, I]) and the
+ * scales into o_sf[t / n_local] (device, h3dit_mx_scale_bytes(n_local, I)
+ * bytes, the layout h3dit_mx_quantize writes), both host arrays of `ranks`
+ * pointers. */
+h3dit_status h3dit_sp_qkv_scatter_mx(h3dit_ctx *ctx, const void *xq, const void *xq_sf,
+                                     int32_t n_local, int32_t block, const float *rope_rows,
+                                     void *const *recv, int32_t ranks, int32_t rank,
+                                     void *cuda_stream);
+h3dit_status h3dit_sp_attention_scatter_mx(h3dit_ctx *ctx, const void *qkv, int32_t n_total,
+                                           void *const *o, void *const *o_sf, int32_t ranks,
+                                           int32_t rank, void *cuda_stream);
+
 /* Peer-memory mapping for the calls above (CUDA IPC; host calls, no kernel).
  * h3dit_ipc_get_handle writes H3DIT_IPC_HANDLE_BYTES bytes that name the
  * allocation holding the device pointer dev_ptr, and *offset_out, dev_ptr's

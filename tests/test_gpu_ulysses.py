@@ -175,6 +175,72 @@ def test_fused_exchange_full_width_4096(P):
     assert torch.equal(got, ref), f"max diff {float((got - ref).abs().max())}"
 
 
+def _run_fused_mx(dims, n_blocks, P, n_txt, grids, seed):
+    """The fused exchanges on an MXFP8 context: each rank quantizes its rows,
+    its QKV (the context's quantized weights) stores into every rank's bf16
+    receive buffer, and its attention writes MXFP8 rows and scales into every
+    rank's out-projection input; compared with the unsharded MXFP8 step."""
+    from image_generation_b200 import h3dit as H
+    from image_generation_b200.ulysses import FusedUlyssesRank
+
+    tw = time_tensors(synth.time_weights(dims, seed))
+    weights = [block_tensors(synth.block_weights(dims, seed + 100 + l)) for l in range(n_blocks)]
+    n_total = n_txt + sum(h * w for _, h, w in grids)
+    cfg = H.make_config(dims.hidden, dims.heads, dims.head_dim, dims.ffn, n_blocks, n_total,
+                        io_fp32=True, precision=H.H3DIT_PRECISION_MXFP8)
+    ctx = H.Context(cfg, tw, weights)
+    ranks = [FusedUlyssesRank(ctx, r, P, n_total, dims.hidden, dims.heads, dims.head_dim,
+                              dims.ffn, mx=True) for r in range(P)]
+    for r in ranks:
+        r.recv.fill_(float("nan"))
+        r.connect([q.recv.data_ptr() for q in ranks], [q.o.data_ptr() for q in ranks],
+                  [q.o_sf.data_ptr() for q in ranks])
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    x = torch.randn(n_total, dims.hidden, device="cuda", generator=g)
+    c = torch.empty(dims.hidden, device="cuda")
+    mod = torch.empty(n_blocks, 6, dims.hidden, device="cuda")
+    rope = torch.empty(n_total, dims.head_dim // 2, 2, device="cuda")
+    ctx.time_embed(0.4, c)
+    ctx.adaln_project(c, 0, n_blocks, mod)
+    ctx.rope_table(grids, n_txt, rope)
+    xs = [x[r.rows()].clone() for r in ranks]
+    for l, w in enumerate(weights):
+        for i, r in enumerate(ranks):
+            r.qkv_scatter(xs[i], mod[l], w, rope[r.rows()], block=l)
+        for r in ranks:
+            r.attention_scatter()
+        for i, r in enumerate(ranks):
+            r.finish(xs[i], mod[l], w, block=l)
+    got = torch.cat(xs)
+    xt, xi = x[:n_txt].clone(), x[n_txt:].clone()
+    ctx.step(0.4, xi, grids, xt)
+    torch.cuda.synchronize()
+    assert ctx.sync_status() == 0
+    ref = torch.cat([xt, xi])
+    assert not torch.equal(ref, x)
+    return got, ref
+
+
+@pytest.mark.parametrize("P", [2, 4, 8])
+def test_fused_exchange_mxfp8_emulated_ranks_small(P):
+    got, ref = _run_fused_mx(synth.SMALL, 2, P, 32, [(0, 16, 16)], 4)
+    assert torch.equal(got, ref), f"max diff {float((got - ref).abs().max())}"
+
+
+def test_fused_exchange_mxfp8_head_dim_128_ragged():
+    dims = synth.Dims(hidden=768, heads=8, head_dim=128, ffn=2048)
+    got, ref = _run_fused_mx(dims, 2, 4, 8, [(0, 32, 37), (1, 4, 2)], 5)
+    assert torch.equal(got, ref), f"max diff {float((got - ref).abs().max())}"
+
+
+def test_fused_exchange_mxfp8_full_width_4096():
+    """SP4 with the MXFP8 linears at full width on the 4096^2 sequence, one
+    block: the pages' latency configuration."""
+    got, ref = _run_fused_mx(synth.FULL_96, 1, 4, 512, [(0, 128, 128)], 6)
+    assert torch.equal(got, ref), f"max diff {float((got - ref).abs().max())}"
+
+
 def test_fused_exchange_writes_only_its_blocks():
     """Every receive and output buffer sits between guard margins; the two
     fused calls of all ranks must fill the buffers and leave the margins."""

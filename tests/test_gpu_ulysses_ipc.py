@@ -1,13 +1,14 @@
-"""Ulysses with the fused exchanges across real processes: 2 and 4 ranks, each
-its own process and CUDA context on cuda:0, map one another's receive and
-output buffers with CUDA IPC (connect_peers: handles exchanged over gloo,
+"""Ulysses with the fused exchanges across real processes: 2 and 4 ranks,
+and 2 with the MXFP8 linears, each its own process and CUDA context on
+cuda:0. They map one another's receive and output buffers (and, in MXFP8, the
+output scales) with CUDA IPC (connect_peers: handles exchanged over gloo,
 h3dit_ipc_open in every other process), run a 2-block step with the host
 barrier after each fused stage (stream synchronise, then a gloo barrier), and
-must reproduce the unsharded step bit for bit. This is the whole multi-process
-path of the fused form - peer mapping, byte offsets inside the caching
-allocator's segments, barriers, unmapping - with the peers on one device.
-No kernel waits on another rank: every rank's kernels only store, and the
-ordering comes from the host barrier."""
+must reproduce the unsharded step bit for bit. This is the whole
+multi-process path of the fused form - peer mapping, byte offsets inside the
+caching allocator's segments, barriers, unmapping - with the peers on one
+device. No kernel waits on another rank: every rank's kernels only store, and
+the ordering comes from the host barrier."""
 import datetime
 import os
 import socket
@@ -19,7 +20,7 @@ pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 
 
-def _rank_main(rank, world, port, out):
+def _rank_main(rank, world, port, mx, out):
     import torch
     import torch.distributed as dist
 
@@ -38,14 +39,15 @@ def _rank_main(rank, world, port, out):
         tw = time_tensors(synth.time_weights(dims, 1))
         weights = [block_tensors(synth.block_weights(dims, 101 + l)) for l in range(n_blocks)]
         cfg = H.make_config(dims.hidden, dims.heads, dims.head_dim, dims.ffn, n_blocks, n_total,
-                            io_fp32=True)
+                            io_fp32=True,
+                            precision=H.H3DIT_PRECISION_MXFP8 if mx else H.H3DIT_PRECISION_BF16)
         ctx = H.Context(cfg, tw, weights)
         g = torch.Generator(device="cuda")
         g.manual_seed(1)
         x = torch.randn(n_total, dims.hidden, device="cuda", generator=g)
         barrier = host_barrier()
         step = UlyssesStep(ctx, weights, rank, world, n_total, dims.hidden, dims.heads,
-                           dims.head_dim, dims.ffn, fused=True, barrier=barrier)
+                           dims.head_dim, dims.ffn, fused=True, barrier=barrier, mx=mx)
         own = step.r.recv_ptrs[rank] == step.r.recv.data_ptr()
         others = len({p for i, p in enumerate(step.r.recv_ptrs) if i != rank}) == world - 1
         xl = x[step.r.rows()].clone()
@@ -77,15 +79,17 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-@pytest.mark.parametrize("world", [2, 4])
-def test_fused_exchange_across_processes_with_ipc(world):
+@pytest.mark.parametrize("world,mx", [(2, False), (4, False), (2, True)],
+                         ids=["sp2", "sp4", "sp2_mxfp8"])
+def test_fused_exchange_across_processes_with_ipc(world, mx):
     import torch.multiprocessing as mp
 
     ctx = mp.get_context("spawn")
     with ctx.Manager() as mgr:
         out = mgr.dict()
         port = _free_port()
-        procs = [ctx.Process(target=_rank_main, args=(r, world, port, out)) for r in range(world)]
+        procs = [ctx.Process(target=_rank_main, args=(r, world, port, mx, out))
+                 for r in range(world)]
         for p in procs:
             p.start()
         for p in procs:
