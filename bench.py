@@ -803,7 +803,7 @@ def denoise_timing(ctx, x_txt, rank, world, barrier, dist, stream, reps: int = 2
                     "h2d_bytes_per_run": in_bytes, "d2h_bytes_per_run": h_out.numel() * 4}}
 
 
-def sp_fused_timing(ctx, block, ranks: int = 4, reps: int = 3) -> dict:
+def sp_fused_timing(ctx, block, ranks: int = 4, reps: int = 3, mx: bool = False) -> dict:
     """One block of the 4096^2 step under Ulysses SP with the fused exchanges,
     all `ranks` ranks on this one GPU: each rank's three stages (RMSNorm +
     QKV storing into every rank's receive buffer; attention of its head group
@@ -811,16 +811,18 @@ def sp_fused_timing(ctx, block, ranks: int = 4, reps: int = 3) -> dict:
     through the library, timed per stage with CUDA events, next to the
     unsharded block. On one GPU the ranks run one after another, so the total
     is the block's whole work plus the decomposition's overhead; the per-rank
-    stage times are what one GPU of an SP group would spend."""
+    stage times are what one GPU of an SP group would spend. With mx the
+    context is MXFP8 and the ranks run its MXFP8 block."""
     import torch
 
     from image_generation_b200.ulysses import FusedUlyssesRank
 
     n_total = N_TOK
-    rs = [FusedUlyssesRank(ctx, r, ranks, n_total, D, H, ctx.cfg.head_dim, F)
+    rs = [FusedUlyssesRank(ctx, r, ranks, n_total, D, H, ctx.cfg.head_dim, F, mx=mx)
           for r in range(ranks)]
     for r in rs:
-        r.connect([q.recv.data_ptr() for q in rs], [q.o.data_ptr() for q in rs])
+        r.connect([q.recv.data_ptr() for q in rs], [q.o.data_ptr() for q in rs],
+                  [q.o_sf.data_ptr() for q in rs] if mx else None)
     c = torch.empty(D, device="cuda")
     mod = torch.empty(1, 6, D, device="cuda")
     rope = torch.empty(n_total, ctx.cfg.head_dim // 2, 2, device="cuda")
@@ -1111,6 +1113,10 @@ def run_h3dit(args):
             ctx_mx = Hb.Context(cfg_mx, tw, blocks)
             ms_mx, prof_mx, launches_mx = time_steps(ctx_mx, args.steps, args.warmup, x_img,
                                                      x_txt, grids, barrier, dist)
+            sp_mx = None
+            if world == 1 and not args.no_sp and dh == 96:
+                sp_mx = optional_leg("sp_fused_mxfp8",
+                                     lambda: sp_fused_timing(ctx_mx, blocks[0], mx=True))
             ctx_mx.close()
             peaks, peak_src = load_peaks()
             fp8_peak = 2.0 * float(peaks["bf16_tflops_sustained"])
@@ -1127,7 +1133,8 @@ def run_h3dit(args):
                     "gemm_frac_of_nominal_fp8": round(g_tf / NOMINAL_FP8_TFLOPS, 4),
                     "kernels": {k: round(v[0] / max(v[1], 1), 4) for k, v in prof_mx.items()
                                 if v[1]},
-                    "gpu_launches": launches_mx}
+                    "gpu_launches": launches_mx,
+                    "ulysses_sp4_fused_one_gpu": sp_mx}
         mx = optional_leg("mxfp8", mxfp8)
         if rank == 0:
             line["mxfp8"] = mx
