@@ -192,6 +192,58 @@ def test_attention(request, which, n, packed):
     assert_attention_bound(to_np(o), ref, float(np.abs(v).max()), "attention")
 
 
+def _rescales_per_row(q, k, d, bkv=64, threshold=8.0):
+    """How often the kernel's running max is replaced (and O rescaled) per
+    query row: the max starts at the first 64-key tile's row max, in log2
+    units, and moves only when a tile's max exceeds it by more than 8."""
+    n, H_ = q.shape[0], q.shape[1]
+    sl2 = np.log2(np.e) / np.sqrt(d)
+    counts = np.zeros((n, H_), np.int64)
+    for h in range(H_):
+        s = (q[:, h].astype(np.float64) @ k[:, h].astype(np.float64).T) * sl2
+        m = s[:, :bkv].max(axis=1)
+        for j in range(bkv, s.shape[1], bkv):
+            mx = s[:, j:j + bkv].max(axis=1)
+            grow = mx > m + threshold
+            counts[grow, h] += 1
+            m = np.where(grow, mx, m)
+    return counts
+
+
+@pytest.mark.parametrize("which", ["small", "small128"])
+@pytest.mark.parametrize("pattern", ["jump", "gradual"])
+def test_attention_running_max_growth(request, which, pattern):
+    """Scores that grow along the key sequence, so that the running max moves
+    by more than 8 (log2 units) and O is rescaled in tensor memory: a shared
+    component in dimension 0 of every head (q + 4, k + 24 from key 500 on:
+    one jump of 12-14 log2 units; or k + 3 t in key tile t: a rescale every
+    few tiles). Without the rescale the early keys would weigh up to 2^8
+    times too much, far outside the bound."""
+    ctx, ocfg, _, _ = request.getfixturevalue(which)
+    H_, d = ocfg.heads, ocfg.head_dim
+    I, n = H_ * d, 1000
+    q = synth.normal_bf16((n, H_, d), 1.0, 11, "q").astype(np.float32)
+    k = synth.normal_bf16((n, H_, d), 1.0, 11, "k").astype(np.float32)
+    v = synth.normal_bf16((n, H_, d), 1.0, 11, "v")
+    q[:, :, 0] += 4.0
+    if pattern == "jump":
+        k[500:, :, 0] += 24.0
+    else:
+        k[:, :, 0] += 3.0 * (np.arange(n) // 64)[:, None]
+    q, k = synth.round_to_bf16(q), synth.round_to_bf16(k)  # the values the GPU sees
+    counts = _rescales_per_row(q, k, d)
+    # the case does what it is for: (almost) every row's O gets rescaled
+    assert (counts >= 1).mean() > 0.9, float((counts >= 1).mean())
+    if pattern == "gradual":
+        assert counts.mean() > 1.5, float(counts.mean())
+    o = torch.empty(n, I, dtype=torch.bfloat16, device="cuda")
+    ctx.attention(to_dev(q.reshape(n, I)), to_dev(k.reshape(n, I)), to_dev(v.reshape(n, I)), I, o,
+                  I, n)
+    _ok(ctx)
+    ref = O.attention(q, k, v).reshape(n, I)
+    assert_attention_bound(to_np(o), ref, float(np.abs(v).max()), f"attention, {pattern} max")
+
+
 def test_attention_identical_keys_give_mean_of_values(small):
     ctx, ocfg, _, _ = small
     n, H_, d = 300, ocfg.heads, ocfg.head_dim
