@@ -273,6 +273,53 @@ def test_fused_exchange_writes_only_its_blocks():
         assert not bool(torch.isnan(b.t.float()).any())
 
 
+def test_fused_exchange_mxfp8_writes_only_its_blocks():
+    """The MXFP8 form's stores (bf16 Q|K|V into the receive buffers, E4M3
+    rows and their scales into the owners' out-projection inputs) stay inside
+    each buffer and fill it: every buffer sits between guard margins. The
+    300-row blocks of each rank end inside a 128-row block of the scale
+    layout."""
+    from image_generation_b200 import h3dit as H
+    from tests.test_gpu_guards import Guarded
+
+    dims, P, n = synth.SMALL, 4, 300
+    n_total = P * n
+    cw, I, D = dims.inner // P, dims.inner, dims.hidden
+    cfg = H.make_config(D, dims.heads, dims.head_dim, dims.ffn, 1, n_total,
+                        precision=H.H3DIT_PRECISION_MXFP8)
+    bw = block_tensors(synth.block_weights(dims, 9))
+    ctx = H.Context(cfg, time_tensors(synth.time_weights(dims, 9)), [bw])
+    recv = [Guarded((n_total, 3 * cw), torch.bfloat16) for _ in range(P)]
+    o = [Guarded((n, I), torch.uint8) for _ in range(P)]
+    o_sf = [Guarded((H.mx_scale_bytes(n, I),), torch.uint8) for _ in range(P)]
+    rope = torch.empty(n_total, dims.head_dim // 2, 2, device="cuda")
+    ctx.rope_table([(0, 30, 40)], 0, rope)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(9)
+    x = torch.randn(n_total, D, device="cuda", generator=g)
+    sh = torch.zeros(D, device="cuda")
+    for r in range(P):
+        xq = torch.empty(n, D, dtype=torch.uint8, device="cuda")
+        xq_sf = torch.empty(H.mx_scale_bytes(n, D), dtype=torch.uint8, device="cuda")
+        ctx.rmsnorm_modulate_mx(x[r * n:(r + 1) * n].contiguous(), sh, sh, xq, xq_sf)
+        ctx.sp_qkv_scatter_mx(xq, xq_sf, 0, rope[r * n:(r + 1) * n],
+                              [b.t.data_ptr() for b in recv], r)
+    for r in range(P):
+        ctx.sp_attention_scatter_mx(recv[r].t, [b.t.data_ptr() for b in o],
+                                    [b.t.data_ptr() for b in o_sf], r)
+    torch.cuda.synchronize()
+    assert ctx.sync_status() == 0
+    for i, b in enumerate(recv):
+        b.check(f"receive buffer {i}")
+        assert not bool(torch.isnan(b.t.float()).any())
+    for i, (b, f) in enumerate(zip(o, o_sf)):
+        b.check(f"E4M3 output {i}")
+        f.check(f"scales {i}")
+        # every code written (0xFF, the fill, is an E4M3 NaN the saturating
+        # quantization never produces); the scale array's padding rows stay
+        assert not bool((b.t == 0xFF).any()), f"E4M3 output {i} not filled"
+
+
 def test_fused_exchange_errors():
     from image_generation_b200 import h3dit as H
 
