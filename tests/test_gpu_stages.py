@@ -72,6 +72,32 @@ def test_rmsnorm_modulate(small, n):
     assert_bf16_rounding(to_np(out), ref, "rmsnorm+modulate")
 
 
+def test_rmsnorm_modulate_extreme_rows(small):
+    """Rows of exact zeros (the epsilon alone sets the scale: the output is
+    the shift), rows near the bottom of fp32 (squares below the smallest
+    normal) and rows near its top (squares summed near 1e33): the kernel's
+    fp32 sum of squares must neither overflow nor flush a row to zero where
+    the float64 oracle does not."""
+    ctx, ocfg, _, _ = small
+    D = ocfg.hidden
+    x = synth.normal_f32((8, D), 1.0, 8, "x")
+    x[0] = 0.0
+    x[1] *= np.float32(1e-20)
+    x[2] *= np.float32(1e15)
+    x[3, :] = 0.0
+    x[3, 5] = np.float32(3e-30)  # a single tiny nonzero
+    sh = synth.normal_f32((D,), 0.3, 8, "shift")
+    sc = synth.normal_f32((D,), 0.3, 8, "scale")
+    out = torch.empty(8, D, dtype=torch.bfloat16, device="cuda")
+    ctx.rmsnorm_modulate(to_dev(x, "f32"), to_dev(sh, "f32"), to_dev(sc, "f32"), out)
+    _ok(ctx)
+    got = to_np(out)
+    ref = O.norm_modulate(x.astype(np.float64), sh, sc, ocfg.norm_eps)
+    assert np.all(np.isfinite(got))
+    assert_bf16_rounding(got, ref, "rmsnorm+modulate, extreme rows")
+    assert np.array_equal(got[0], to_np(to_dev(sh)))  # zero row: exactly the shift in bf16
+
+
 @pytest.mark.parametrize("grids,n_txt", [([(0, 16, 16)], 32), ([(0, 5, 7), (1, 3, 4), (3, 2, 9)], 3),
                                          ([(0, 128, 128)], 512)])
 @pytest.mark.parametrize("which", ["small", "small128"])
