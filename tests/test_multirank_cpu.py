@@ -61,3 +61,25 @@ def test_reference_arm_runs_only_on_rank_zero(monkeypatch):
     args = type("A", (), {"warmup": 1, "steps": 1, "head_dim": 96, "gpus": 2})()
     assert bench.run_reference(args) == 0
     assert not called
+
+
+def test_streaming_placements():
+    """The weight-streaming leg's two placements: "tail" streams the last
+    L - k blocks; "spread" streams as many, spaced evenly, so that no two
+    streamed blocks are adjacent while at least half the blocks stay
+    resident, and no gap between streamed blocks exceeds one block more than
+    the even spacing."""
+    import bench
+
+    L = bench.L
+    for k in range(L + 1):
+        tail = bench.streamed_set(k, "tail")
+        spread = bench.streamed_set(k, "spread")
+        assert tail == set(range(k, L))
+        assert len(spread) == L - k and spread <= set(range(L))
+        idx = sorted(spread)
+        if 2 * k >= L:
+            assert all(b - a >= 2 for a, b in zip(idx, idx[1:])), k
+        if len(idx) > 1:
+            gaps = [b - a for a, b in zip(idx, idx[1:])]
+            assert max(gaps) - min(gaps) <= 1, (k, gaps)
